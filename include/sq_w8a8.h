@@ -1,0 +1,187 @@
+/*
+ * sq_w8a8.h -- C ABI of the SmoothQuant W8A8 linear layer with a
+ * per-request LoRA delta, for NVIDIA B200 (sm_100a).
+ *
+ * What it computes (sources named by page title and section):
+ *  - "SmoothQuant" explainer (ozercemkelahmet.com/tools/smoothquant),
+ *    How it works, Steps 2-7, and its Python sketch: per-channel smoothing
+ *    s_j = max|X_j|^alpha / max|W_j|^(1-alpha), folded into the weights;
+ *    per-token dynamic INT8 activations; per-output-channel INT8 weights;
+ *    INT8 x INT8 GEMM with INT32 accumulation, dequantized with the stored
+ *    scales.
+ *  - "[Feature]: LoRA support for W8A8 SmoothQuant" (TensorRT-LLM issue
+ *    #12703), Pitch: a BF16 low-rank LoRA path after the INT8 GEMM whose
+ *    result is added to the dequantized output; Motivation: one adapter per
+ *    request, many requests per batch.
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, row-major,
+ *    16-byte aligned.  The library never allocates device memory.
+ *  - bf16 tensors are passed as uint16_t bit patterns.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *    only enqueue work: they return after validating arguments and
+ *    launching, and the results are ready when the stream reaches them.
+ *  - Return value: SQ_OK (0) or an sq_status code.  Argument errors are found
+ *    on the host before anything is launched and leave the outputs untouched.
+ *    Errors found on the device (a wait that ran out, a segment naming an
+ *    adapter that does not exist) do not fault: the kernel records a code
+ *    that sq_get_device_error() returns.
+ *  - Only compute capability 10.0 (B200) is supported; other devices get
+ *    SQ_ERR_UNSUPPORTED_DEVICE.  There is no fallback path.
+ *
+ * Shapes: M tokens, K input channels, N output channels.
+ *   X  [M,K]  bf16 or f32        Xq [M,K] int8      x_scale [M] f32
+ *   W  [N,K]  bf16 (torch Linear layout: output channels by input channels)
+ *   Wq [N,K]  int8               w_scale [N] f32    s [K] f32
+ *   Y  [M,N]  bf16
+ * Constraints: K % 16 == 0, N % 16 == 0, K <= SQ_MAX_K (a row of K fp32
+ * values is staged in shared memory; K*127^2 then also fits in int32).
+ */
+#ifndef SQ_W8A8_H
+#define SQ_W8A8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sq_status {
+  SQ_OK = 0,
+  SQ_ERR_INVALID_ARG = 1,        /* null/misaligned pointer, negative size  */
+  SQ_ERR_UNSUPPORTED_SHAPE = 2,  /* K or N not a multiple of 16, K too big  */
+  SQ_ERR_UNSUPPORTED_DEVICE = 3, /* not compute capability 10.0             */
+  SQ_ERR_CUDA = 4,               /* a CUDA runtime call failed              */
+  SQ_ERR_DEVICE_TIMEOUT = 5,     /* a bounded device-side wait ran out      */
+  SQ_ERR_WORKSPACE = 6,          /* workspace missing or too small          */
+  SQ_ERR_BAD_SEGMENTS = 7        /* device: adapter index out of range      */
+} sq_status;
+
+typedef enum sq_dtype { SQ_DTYPE_F32 = 0, SQ_DTYPE_BF16 = 1 } sq_dtype;
+
+/* Largest supported number of input channels. */
+#define SQ_MAX_K 57344
+
+/* Largest packed LoRA width (sum over adapters of the rank rounded up to 16). */
+#define SQ_MAX_LORA_COLS 1024
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *sq_status_string(int status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int sq_version(void);
+
+/* SQ_OK if `device` is a compute capability 10.0 GPU, else
+ * SQ_ERR_UNSUPPORTED_DEVICE (or SQ_ERR_CUDA if it cannot be queried). */
+int sq_device_supported(int device);
+
+/* Device-side error code recorded by earlier launches on the current device
+ * (an sq_status value, 0 if none), after synchronizing the device.  If
+ * `clear` is nonzero the record is reset to 0. */
+int sq_get_device_error(int *code, int clear);
+
+/* Upper bound, in nanoseconds, of every spin-wait inside the kernels
+ * (default 2 s).  A wait that runs out makes the kernel stop, record
+ * SQ_ERR_DEVICE_TIMEOUT and return.  Host-side setting for later launches. */
+int sq_set_wait_timeout_ns(uint64_t ns);
+
+/* ---------------------------------------------------------------------------
+ * Offline preparation ("SmoothQuant" explainer, Steps 3-5 and the sketch)
+ * ------------------------------------------------------------------------ */
+
+/* Calibration ("Calibration in practice"): act_absmax[j] =
+ * max(act_absmax[j], max_i |X[i,j]|).  X [M,K] of x_dtype; act_absmax [K]
+ * f32, read and written (zero it before the first batch). */
+int sq_act_absmax_update(const void *X, int x_dtype, int64_t M, int64_t K,
+                         float *act_absmax, void *stream);
+
+/* w_absmax[j] = max_n |W[n,j]| (the sketch's abs().max(dim=0) over the
+ * output channels).  W [N,K] bf16; w_absmax [K] f32, written. */
+int sq_weight_absmax(const uint16_t *W, int64_t N, int64_t K, float *w_absmax,
+                     void *stream);
+
+/* Step 3 and the sketch: s_j = max(max(a_j,1e-5)^alpha /
+ * max(w_j,1e-5)^(1-alpha), 1e-5), evaluated in fp64 and rounded once to fp32.
+ * act_absmax, w_absmax, s: [K] f32. alpha in [0,1]. */
+int sq_compute_smoothing(const float *act_absmax, const float *w_absmax, int64_t K,
+                         float alpha, float *s, void *stream);
+
+/* Steps 5-6: fold s into the weights along the input channels and quantize
+ * each output channel:  W' = fp32(W[n,k]*s_k);  w_scale_n = max_k|W'|/127;
+ * Wq = clamp(round_half_even(W'/w_scale_n), -128, 127)  (IEEE fp32 division;
+ * an all-zero channel gets scale 0 and codes 0).  Bit-exact. */
+int sq_quantize_weight(const uint16_t *W, const float *s, int64_t N, int64_t K,
+                       int8_t *Wq, float *w_scale, void *stream);
+
+/* LoRA adapter table.  Adapters are packed side by side: adapter a of rank
+ * r_a owns columns [off_a, off_a + round_up(r_a,16)) of the packed width
+ * R = sum_a round_up(r_a,16) <= SQ_MAX_LORA_COLS, in
+ *   A_pack [R, K] bf16 : rows off_a+j   = bf16(fp32(A_a[j,k] * s_k))
+ *   B_pack [N, R] bf16 : cols off_a+j   = bf16(fp32(B_a[n,j] * lora_alpha/r))
+ * with zeros in the padding rows/columns.  Folding s into A lets the LoRA
+ * path read the dequantized activations Xq*x_scale (which approximate X/s)
+ * and still compute X*A^T; folding lora_alpha/r into B applies the LoRA
+ * scaling once, offline.  This call writes adapter (A [r,K], B [N,r], both
+ * bf16) at column offset `off` (a multiple of 16) of a pack of width R. */
+int sq_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s, int64_t r,
+                    int64_t K, int64_t N, float lora_alpha, int64_t R, int64_t off,
+                    uint16_t *A_pack, uint16_t *B_pack, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Hot path
+ * ------------------------------------------------------------------------ */
+
+/* Steps 2 and 6 (dynamic per-token scales): divide each channel by s_j, then
+ * quantize each token:  xt = fp32(X[i,j]/s_j);  x_scale_i = max_j|xt|/127;
+ * Xq = clamp(round_half_even(xt/x_scale_i), -128, 127), all divisions IEEE
+ * fp32 (an all-zero token gets scale 0 and codes 0).  Bit-exact.
+ * X [M,K] of x_dtype (SQ_DTYPE_BF16 or SQ_DTYPE_F32). */
+int sq_quant_act(const void *X, int x_dtype, const float *s, int64_t M, int64_t K,
+                 int8_t *Xq, float *x_scale, void *stream);
+
+/* Bytes of device workspace sq_linear_lora needs for M tokens and a LoRA
+ * pack of width R (0 when R == 0). */
+size_t sq_linear_lora_workspace_size(int64_t M, int64_t R);
+
+/* Step 7 plus the LoRA delta, one launch sequence:
+ *   Y[i,n] = bf16( f32(acc[i,n]) * x_scale_i * w_scale_n + delta[i,n] ),
+ *   acc = Xq Wq^T (exact int32), delta[i,:] = (x_scale_i Xq[i,:] A_pack_a^T)
+ *   B_pack_a^T for the adapter a of token i (none: delta = 0).
+ * Segments: seg_offsets [S+1] and seg_adapter [S] (device int32): token i
+ * belongs to the first segment s with seg_offsets[s] <= i < seg_offsets[s+1]
+ * and uses adapter seg_adapter[s]; -1 (or no segment) means no LoRA.  An
+ * adapter index >= n_adapters is treated as -1 and recorded as
+ * SQ_ERR_BAD_SEGMENTS.  lora_offset / lora_rank: [n_adapters] device int32
+ * (column offset and rank of each adapter in the pack).  With R == 0,
+ * n_adapters == 0 or S == 0 the layer is plain W8A8 and the LoRA arguments
+ * may be NULL.  workspace: >= sq_linear_lora_workspace_size(M, R) bytes of
+ * device memory, 256-byte aligned; its contents are scratch. */
+int sq_linear_lora(const int8_t *Xq, const float *x_scale, const int8_t *Wq,
+                   const float *w_scale, int64_t M, int64_t N, int64_t K,
+                   const uint16_t *A_pack, const uint16_t *B_pack,
+                   const int32_t *lora_offset, const int32_t *lora_rank, int n_adapters,
+                   int64_t R, const int32_t *seg_offsets, const int32_t *seg_adapter,
+                   int64_t S, uint16_t *Y, void *workspace, size_t workspace_bytes,
+                   void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Test entries: the same kernels with a different epilogue
+ * ------------------------------------------------------------------------ */
+
+/* acc [M,N] int32 = Xq Wq^T exactly (the INT32 accumulators of Step 7). */
+int sq_gemm_i32(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N, int64_t K,
+                int32_t *acc, void *stream);
+
+/* delta [M,N] f32: the LoRA delta alone, as sq_linear_lora adds it. */
+int sq_lora_delta(const int8_t *Xq, const float *x_scale, int64_t M, int64_t N,
+                  int64_t K, const uint16_t *A_pack, const uint16_t *B_pack,
+                  const int32_t *lora_offset, const int32_t *lora_rank, int n_adapters,
+                  int64_t R, const int32_t *seg_offsets, const int32_t *seg_adapter,
+                  int64_t S, float *delta, void *workspace, size_t workspace_bytes,
+                  void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SQ_W8A8_H */

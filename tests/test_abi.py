@@ -1,0 +1,109 @@
+"""The C ABI library loads without a GPU, exports every entry point that
+include/sq_w8a8.h declares, and rejects bad arguments on the host before any
+launch (no compute call is made here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from w8a8_smoothquant_int8_b200 import _native, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "sq_w8a8.h")
+
+OK, INVALID, SHAPE, DEVICE, CUDA, TIMEOUT, WORKSPACE, SEGMENTS = range(8)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _native.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("sq_compute_smoothing", "sq_quantize_weight", "sq_quant_act", "sq_linear_lora"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _native.SIGNATURES, n
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        assert lib.sq_status_string(code)
+    assert b"unknown" in lib.sq_status_string(99)
+    assert lib.sq_version() >= 100
+
+
+def test_workspace_size(lib):
+    assert lib.sq_linear_lora_workspace_size(2048, 0) == 0
+    assert lib.sq_linear_lora_workspace_size(0, 16) == 0
+    ws = lib.sq_linear_lora_workspace_size(2048, 16)
+    assert ws >= 2 * 2048 * 16 * 2 + 16 * 8 and ws % 256 == 0
+
+
+A = 1 << 20  # a 16-byte-aligned fake address: never dereferenced, validation fails first
+
+
+def test_quant_act_validation(lib):
+    f = lib.sq_quant_act
+    assert f(A, 1, A, 4, 15, A, A, None) == SHAPE          # K % 16
+    assert f(A, 1, A, 4, 57344 + 16, A, A, None) == SHAPE  # K too large
+    assert f(A, 1, A, -1, 16, A, A, None) == INVALID       # negative M
+    assert f(A, 7, A, 4, 16, A, A, None) == INVALID        # dtype
+    assert f(A + 8, 1, A, 4, 16, A, A, None) == INVALID    # misaligned X
+    assert f(None, 1, A, 4, 16, A, A, None) == INVALID     # null X
+    # well-formed arguments reach the device check: no device here
+    assert f(A, 1, A, 4, 16, A, A, None) in (CUDA, DEVICE)
+
+
+def test_linear_lora_validation(lib):
+    f = lib.sq_linear_lora
+    ws = lib.sq_linear_lora_workspace_size(256, 32)
+    args = dict(Xq=A, xs=A, Wq=A, ws_=A, M=256, N=512, K=1024, Ap=A, Bp=A, off=A, rk=A, nad=2, R=32,
+                so=A, sa=A, S=3, Y=A, w=A, wb=ws, st=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return f(a["Xq"], a["xs"], a["Wq"], a["ws_"], a["M"], a["N"], a["K"], a["Ap"], a["Bp"], a["off"],
+                 a["rk"], a["nad"], a["R"], a["so"], a["sa"], a["S"], a["Y"], a["w"], a["wb"], a["st"])
+
+    assert call(N=100) == SHAPE               # N % 16
+    assert call(K=1000) == SHAPE              # K % 16
+    assert call(R=24) == SHAPE                # R % 16
+    assert call(R=2048) == SHAPE              # R > 1024
+    assert call(nad=-1) == INVALID
+    assert call(wb=ws - 1) == WORKSPACE
+    assert call(w=A + 16) == WORKSPACE        # workspace must be 256-byte aligned
+    assert call(w=None) == WORKSPACE
+    assert call(Bp=None) == INVALID
+    assert call(Y=A + 4) == INVALID
+    assert call() in (CUDA, DEVICE)
+    # no LoRA: the LoRA pointers and the workspace may be null
+    assert call(R=0, Ap=None, Bp=None, off=None, rk=None, so=None, sa=None, S=0, w=None, wb=0) in (CUDA, DEVICE)
+
+
+def test_offline_validation(lib):
+    assert lib.sq_compute_smoothing(A, A, 64, 1.5, A, None) == INVALID
+    assert lib.sq_compute_smoothing(A, A, 64, -0.1, A, None) == INVALID
+    assert lib.sq_quantize_weight(A, A, 8, 24, A, A, None) == SHAPE
+    assert lib.sq_prepare_lora(A, A, A, 8, 64, 32, 16.0, 16, 8, A, A, None) == SHAPE   # off % 16
+    assert lib.sq_prepare_lora(A, A, A, 20, 64, 32, 16.0, 16, 0, A, A, None) == INVALID  # r > R
+    assert lib.sq_prepare_lora(A, A, A, 0, 64, 32, 16.0, 16, 0, A, A, None) == INVALID
+    assert lib.sq_set_wait_timeout_ns(0) == INVALID
+    code = ctypes.c_int(0)
+    assert lib.sq_get_device_error(None, 0) == INVALID

@@ -1,0 +1,260 @@
+// C ABI entry points (include/sq_w8a8.h): argument validation on the host,
+// then launches.  Nothing here allocates device memory.
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+
+namespace sq {
+
+static uint64_t g_wait_timeout_ns = 2000000000ull;
+uint64_t wait_timeout_ns() { return g_wait_timeout_ns; }
+
+// ---------------------------------------------------------------------------
+// validation helpers
+// ---------------------------------------------------------------------------
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool ptr_ok(const void *p) { return p != nullptr && aligned16(p); }
+
+static int check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SQ_ERR_CUDA;
+  return sq_device_supported(dev);
+}
+
+static int check_mk(int64_t M, int64_t K) {
+  if (M < 0 || K < 0) return SQ_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K > SQ_MAX_K) return SQ_ERR_UNSUPPORTED_SHAPE;
+  if (M > 0x7fffffffLL) return SQ_ERR_UNSUPPORTED_SHAPE;
+  return SQ_OK;
+}
+
+static int cuda_status(cudaError_t e) { return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA; }
+
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct Workspace {
+  uint16_t *T_hi, *T_lo;
+  unsigned long long *mask;
+};
+
+static size_t workspace_bytes(int64_t M, int64_t R) {
+  if (R <= 0 || M <= 0) return 0;
+  const size_t plane = align256(static_cast<size_t>(M) * static_cast<size_t>(R) * 2);
+  return 2 * plane + align256(static_cast<size_t>((M + 127) / 128) * 8);
+}
+
+static Workspace carve(void *ws, int64_t M, int64_t R) {
+  const size_t plane = align256(static_cast<size_t>(M) * static_cast<size_t>(R) * 2);
+  uint8_t *p = static_cast<uint8_t *>(ws);
+  return Workspace{reinterpret_cast<uint16_t *>(p), reinterpret_cast<uint16_t *>(p + plane),
+                   reinterpret_cast<unsigned long long *>(p + 2 * plane)};
+}
+
+// checks shared by sq_linear_lora and sq_lora_delta
+static int check_lora_args(int64_t M, int64_t K, const uint16_t *A_pack, const uint16_t *B_pack,
+                           const int32_t *lora_offset, const int32_t *lora_rank, int n_adapters,
+                           int64_t R, const int32_t *seg_offsets, const int32_t *seg_adapter,
+                           int64_t S, void *workspace, size_t workspace_size, bool *active) {
+  if (n_adapters < 0 || R < 0 || S < 0) return SQ_ERR_INVALID_ARG;
+  *active = (R > 0 && n_adapters > 0 && S > 0 && M > 0);
+  if (!*active) return SQ_OK;
+  if (R % 16 != 0 || R > SQ_MAX_LORA_COLS) return SQ_ERR_UNSUPPORTED_SHAPE;
+  if (!ptr_ok(A_pack) || !ptr_ok(B_pack) || !lora_offset || !lora_rank || !seg_offsets ||
+      !seg_adapter)
+    return SQ_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_size < workspace_bytes(M, R))
+    return SQ_ERR_WORKSPACE;
+  (void)K;
+  return SQ_OK;
+}
+
+}  // namespace sq
+
+using namespace sq;
+
+extern "C" {
+
+const char *sq_status_string(int status) {
+  switch (status) {
+    case SQ_OK: return "ok";
+    case SQ_ERR_INVALID_ARG: return "invalid argument";
+    case SQ_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case SQ_ERR_UNSUPPORTED_DEVICE: return "unsupported device (needs compute capability 10.0)";
+    case SQ_ERR_CUDA: return "CUDA runtime error";
+    case SQ_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case SQ_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case SQ_ERR_BAD_SEGMENTS: return "segment table names an adapter that does not exist";
+    default: return "unknown status";
+  }
+}
+
+int sq_version(void) { return 100; }
+
+int sq_device_supported(int device) {
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return SQ_ERR_CUDA;
+  return (prop.major == 10 && prop.minor == 0) ? SQ_OK : SQ_ERR_UNSUPPORTED_DEVICE;
+}
+
+int sq_get_device_error(int *code, int clear) {
+  if (!code) return SQ_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return SQ_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof v) != cudaSuccess) return SQ_ERR_CUDA;
+  *code = static_cast<int>(v);
+  if (clear) {
+    unsigned int z = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &z, sizeof z) != cudaSuccess) return SQ_ERR_CUDA;
+  }
+  return SQ_OK;
+}
+
+int sq_set_wait_timeout_ns(uint64_t ns) {
+  if (ns == 0) return SQ_ERR_INVALID_ARG;
+  g_wait_timeout_ns = ns;
+  return SQ_OK;
+}
+
+int sq_act_absmax_update(const void *X, int x_dtype, int64_t M, int64_t K, float *act_absmax,
+                         void *stream) {
+  int st = check_mk(M, K);
+  if (st) return st;
+  if (x_dtype != SQ_DTYPE_BF16 && x_dtype != SQ_DTYPE_F32) return SQ_ERR_INVALID_ARG;
+  if ((M > 0 && K > 0) && (!ptr_ok(X) || !ptr_ok(act_absmax))) return SQ_ERR_INVALID_ARG;
+  if ((st = check_device())) return st;
+  return cuda_status(launch_act_absmax_update(X, x_dtype, M, K, act_absmax,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+int sq_weight_absmax(const uint16_t *W, int64_t N, int64_t K, float *w_absmax, void *stream) {
+  int st = check_mk(N, K);
+  if (st) return st;
+  if (K > 0 && (!ptr_ok(w_absmax) || (N > 0 && !ptr_ok(W)))) return SQ_ERR_INVALID_ARG;
+  if ((st = check_device())) return st;
+  if (K == 0) return SQ_OK;
+  return cuda_status(launch_weight_absmax(W, N, K, w_absmax, static_cast<cudaStream_t>(stream)));
+}
+
+int sq_compute_smoothing(const float *act_absmax, const float *w_absmax, int64_t K, float alpha,
+                         float *s, void *stream) {
+  if (K < 0) return SQ_ERR_INVALID_ARG;
+  if (!(alpha >= 0.f && alpha <= 1.f)) return SQ_ERR_INVALID_ARG;
+  if (K > 0 && (!ptr_ok(act_absmax) || !ptr_ok(w_absmax) || !ptr_ok(s))) return SQ_ERR_INVALID_ARG;
+  int st = check_device();
+  if (st) return st;
+  return cuda_status(
+      launch_compute_smoothing(act_absmax, w_absmax, K, alpha, s, static_cast<cudaStream_t>(stream)));
+}
+
+int sq_quantize_weight(const uint16_t *W, const float *s, int64_t N, int64_t K, int8_t *Wq,
+                       float *w_scale, void *stream) {
+  int st = check_mk(N, K);
+  if (st) return st;
+  if (N > 0 && (!ptr_ok(w_scale) || (K > 0 && (!ptr_ok(W) || !ptr_ok(s) || !ptr_ok(Wq)))))
+    return SQ_ERR_INVALID_ARG;
+  if ((st = check_device())) return st;
+  return cuda_status(launch_quantize_weight(W, s, N, K, Wq, w_scale, static_cast<cudaStream_t>(stream)));
+}
+
+int sq_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s, int64_t r, int64_t K,
+                    int64_t N, float lora_alpha, int64_t R, int64_t off, uint16_t *A_pack,
+                    uint16_t *B_pack, void *stream) {
+  if (r <= 0 || K < 0 || N < 0 || R <= 0 || off < 0) return SQ_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K > SQ_MAX_K || R % 16 != 0 || R > SQ_MAX_LORA_COLS || off % 16 != 0)
+    return SQ_ERR_UNSUPPORTED_SHAPE;
+  const int64_t rpad = (r + 15) / 16 * 16;
+  if (off + rpad > R) return SQ_ERR_INVALID_ARG;
+  if (!A || !B || !ptr_ok(s) || !ptr_ok(A_pack) || !ptr_ok(B_pack)) return SQ_ERR_INVALID_ARG;
+  int st = check_device();
+  if (st) return st;
+  const float scale = lora_alpha / static_cast<float>(r);  // IEEE fp32 division
+  return cuda_status(launch_prepare_lora(A, B, s, r, K, N, scale, R, off, A_pack, B_pack,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+int sq_quant_act(const void *X, int x_dtype, const float *s, int64_t M, int64_t K, int8_t *Xq,
+                 float *x_scale, void *stream) {
+  int st = check_mk(M, K);
+  if (st) return st;
+  if (x_dtype != SQ_DTYPE_BF16 && x_dtype != SQ_DTYPE_F32) return SQ_ERR_INVALID_ARG;
+  if (M > 0 && (!ptr_ok(x_scale) || (K > 0 && (!ptr_ok(X) || !ptr_ok(s) || !ptr_ok(Xq)))))
+    return SQ_ERR_INVALID_ARG;
+  if ((st = check_device())) return st;
+  return cuda_status(
+      launch_quant_act(X, x_dtype, s, M, K, Xq, x_scale, static_cast<cudaStream_t>(stream)));
+}
+
+size_t sq_linear_lora_workspace_size(int64_t M, int64_t R) { return workspace_bytes(M, R); }
+
+static int linear_common(const int8_t *Xq, const float *x_scale, const int8_t *Wq,
+                         const float *w_scale, int64_t M, int64_t N, int64_t K,
+                         const uint16_t *A_pack, const uint16_t *B_pack,
+                         const int32_t *lora_offset, const int32_t *lora_rank, int n_adapters,
+                         int64_t R, const int32_t *seg_offsets, const int32_t *seg_adapter,
+                         int64_t S, int mode, void *out, void *workspace, size_t workspace_size,
+                         void *stream) {
+  int st = check_mk(M, K);
+  if (st) return st;
+  if (N < 0) return SQ_ERR_INVALID_ARG;
+  if (N % 16 != 0) return SQ_ERR_UNSUPPORTED_SHAPE;
+  bool lora = false;
+  if (mode != 1) {
+    st = check_lora_args(M, K, A_pack, B_pack, lora_offset, lora_rank, n_adapters, R, seg_offsets,
+                         seg_adapter, S, workspace, workspace_size, &lora);
+    if (st) return st;
+  }
+  if (M == 0 || N == 0) return check_device();
+  if (!ptr_ok(out)) return SQ_ERR_INVALID_ARG;
+  if (K > 0 && (!ptr_ok(Xq) || (mode != 2 && !ptr_ok(Wq)))) return SQ_ERR_INVALID_ARG;
+  if (mode != 1 && !ptr_ok(x_scale)) return SQ_ERR_INVALID_ARG;
+  if (mode == 0 && !ptr_ok(w_scale)) return SQ_ERR_INVALID_ARG;
+  if ((st = check_device())) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t esize = (mode == 0) ? 2 : 4;
+  if (K == 0 || (mode == 2 && !lora)) {
+    // empty contraction (and no LoRA rows with K == 0 either: T = 0)
+    return cuda_status(cudaMemsetAsync(out, 0, static_cast<size_t>(M) * N * esize, s));
+  }
+  LoraOperands lo;
+  LoraOperands *lop = nullptr;
+  if (lora) {
+    Workspace w = carve(workspace, M, R);
+    cudaError_t e = launch_lora_shrink(Xq, x_scale, M, K, A_pack, lora_offset, lora_rank,
+                                       n_adapters, R, seg_offsets, seg_adapter, S, w.T_hi, w.T_lo,
+                                       w.mask, s);
+    if (e != cudaSuccess) return SQ_ERR_CUDA;
+    lo = LoraOperands{w.T_hi, w.T_lo, B_pack, w.mask, R};
+    lop = &lo;
+  }
+  return cuda_status(launch_w8a8_gemm(Xq, Wq, x_scale, w_scale, M, N, K, mode, out, lop, s));
+}
+
+int sq_linear_lora(const int8_t *Xq, const float *x_scale, const int8_t *Wq, const float *w_scale,
+                   int64_t M, int64_t N, int64_t K, const uint16_t *A_pack, const uint16_t *B_pack,
+                   const int32_t *lora_offset, const int32_t *lora_rank, int n_adapters, int64_t R,
+                   const int32_t *seg_offsets, const int32_t *seg_adapter, int64_t S, uint16_t *Y,
+                   void *workspace, size_t workspace_size, void *stream) {
+  return linear_common(Xq, x_scale, Wq, w_scale, M, N, K, A_pack, B_pack, lora_offset, lora_rank,
+                       n_adapters, R, seg_offsets, seg_adapter, S, 0, Y, workspace, workspace_size,
+                       stream);
+}
+
+int sq_gemm_i32(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N, int64_t K, int32_t *acc,
+                void *stream) {
+  return linear_common(Xq, nullptr, Wq, nullptr, M, N, K, nullptr, nullptr, nullptr, nullptr, 0, 0,
+                       nullptr, nullptr, 0, 1, acc, nullptr, 0, stream);
+}
+
+int sq_lora_delta(const int8_t *Xq, const float *x_scale, int64_t M, int64_t N, int64_t K,
+                  const uint16_t *A_pack, const uint16_t *B_pack, const int32_t *lora_offset,
+                  const int32_t *lora_rank, int n_adapters, int64_t R, const int32_t *seg_offsets,
+                  const int32_t *seg_adapter, int64_t S, float *delta, void *workspace,
+                  size_t workspace_size, void *stream) {
+  return linear_common(Xq, x_scale, nullptr, nullptr, M, N, K, A_pack, B_pack, lora_offset,
+                       lora_rank, n_adapters, R, seg_offsets, seg_adapter, S, 2, delta, workspace,
+                       workspace_size, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,89 @@
+// Shared definitions of the CUDA library (not part of the public ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/sq_w8a8.h"
+
+namespace sq {
+
+// Device-side error record: the first sq_status code a kernel hits.  The
+// library is built as one translation unit (sq_lib.cu), so this is one object.
+__device__ unsigned int g_device_error = 0;
+
+__device__ __forceinline__ void record_device_error(unsigned int code) {
+  atomicCAS(&g_device_error, 0u, code);
+}
+
+// Default bound of every device-side spin-wait (ns), settable from the host.
+uint64_t wait_timeout_ns();
+
+// LoRA operands of the fused GEMM: T planes [M,R] bf16 (written by the
+// shrink kernel), the packed B [N,R] bf16 and one 16-column-group mask per
+// 128-token tile.
+struct LoraOperands {
+  const uint16_t *T_hi, *T_lo, *B_pack;
+  const unsigned long long *mask;
+  int64_t R;
+};
+
+// launchers (one per kernel family); they only enqueue work on `st`
+cudaError_t launch_act_absmax_update(const void *X, int dtype, int64_t M, int64_t K, float *out,
+                                     cudaStream_t st);
+cudaError_t launch_weight_absmax(const uint16_t *W, int64_t N, int64_t K, float *out,
+                                 cudaStream_t st);
+cudaError_t launch_compute_smoothing(const float *a, const float *w, int64_t K, float alpha,
+                                     float *s, cudaStream_t st);
+cudaError_t launch_quant_act(const void *X, int dtype, const float *s, int64_t M, int64_t K,
+                             int8_t *Xq, float *x_scale, cudaStream_t st);
+cudaError_t launch_quantize_weight(const uint16_t *W, const float *s, int64_t N, int64_t K,
+                                   int8_t *Wq, float *w_scale, cudaStream_t st);
+cudaError_t launch_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s, int64_t r,
+                                int64_t K, int64_t N, float scale, int64_t R, int64_t off,
+                                uint16_t *A_pack, uint16_t *B_pack, cudaStream_t st);
+cudaError_t launch_lora_shrink(const int8_t *Xq, const float *x_scale, int64_t M, int64_t K,
+                               const uint16_t *A_pack, const int32_t *lora_offset,
+                               const int32_t *lora_rank, int n_adapters, int64_t R,
+                               const int32_t *seg_offsets, const int32_t *seg_adapter, int64_t S,
+                               uint16_t *T_hi, uint16_t *T_lo, unsigned long long *mask,
+                               cudaStream_t st);
+cudaError_t launch_w8a8_gemm(const int8_t *Xq, const int8_t *Wq, const float *x_scale,
+                             const float *w_scale, int64_t M, int64_t N, int64_t K, int mode,
+                             void *out, const LoraOperands *lora, cudaStream_t st);
+
+// Adapter of token `i` for a segment table: the first segment s with
+// off[s] <= i < off[s+1].  Segments are assumed sorted (off non-decreasing);
+// the binary search finds the last segment starting at or before i and then
+// checks that it covers i.  Returns -1 when no segment covers the token; an
+// adapter index outside [-1, n_adapters) is reported and treated as -1.
+__device__ __forceinline__ int token_adapter(const int32_t *__restrict__ seg_offsets,
+                                             const int32_t *__restrict__ seg_adapter,
+                                             int64_t S, int n_adapters, int64_t i) {
+  if (S <= 0) return -1;
+  int64_t lo = 0, hi = S - 1, s = -1;
+  while (lo <= hi) {
+    int64_t mid = (lo + hi) >> 1;
+    if (seg_offsets[mid] <= i) {
+      s = mid;
+      lo = mid + 1;
+    } else {
+      hi = mid - 1;
+    }
+  }
+  // several empty segments may start at the same offset: step back to the
+  // first segment whose range is non-empty and holds i
+  while (s >= 0 && !(seg_offsets[s] <= i && i < seg_offsets[s + 1])) {
+    if (seg_offsets[s] < i) return -1;
+    --s;
+  }
+  if (s < 0) return -1;
+  int a = seg_adapter[s];
+  if (a < -1 || a >= n_adapters) {
+    record_device_error(SQ_ERR_BAD_SEGMENTS);
+    return -1;
+  }
+  return a;
+}
+
+}  // namespace sq
