@@ -1,0 +1,383 @@
+#!/usr/bin/env python
+"""Benchmark of the SmoothQuant W8A8 + per-request LoRA linear on B200.
+
+One step = one pass of the whole hot path over one batch: sq_quant_act
+(smoothing + per-token INT8) followed by sq_linear_lora (LoRA shrink, then
+the fused INT8 GEMM + dequant + LoRA delta), on the Llama-3-8B fused QKV
+projection workload (M=2048 tokens, K=4096, N=6144, one rank-16 adapter).
+
+Timing: W untimed warm-up steps, then K timed steps.  Before every step a
+256 MiB buffer is written (untimed) so that L2 (126 MB) holds none of the
+step's inputs; each step is bracketed by CUDA events on the stream the
+kernels run on, and the fused GEMM launch by its own event pair (recorded by
+the library).  Multi-GPU runs are independent replicas (the layer has no
+exchange step): each rank runs the same workload, times are maxed over ranks
+and the throughput counts all ranks' work.
+
+--impl reference times the CPU oracle (fp64/int64 C, OpenMP) on the host
+cores for the same workload and metric, one bounded sample of tokens per step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from w8a8_smoothquant_int8_b200 import workloads as wk  # noqa: E402
+
+METRIC = "W8A8+LoRA linear INT8 TOPS & tokens/s; % of INT8 tensor peak / HBM roofline"
+DEFAULT_WORKLOAD = "llama3_8b_qkv_m2048_k4096_n6144"
+FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wk.SPECS))
+    p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def lora_flops(wl) -> int:
+    ad = wk.row_adapter(wl.seg_offsets, wl.seg_adapter, wl.M, len(wl.adapters))
+    r = np.array([wl.adapters[a].r if a >= 0 else 0 for a in ad], np.int64)
+    return int(2 * r.sum() * (wl.K + wl.N))
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.path = tempfile.mktemp(prefix="sq_clocks_", suffix=".csv")
+        self.proc = None
+        self.gpu = gpu_index
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), max=float(parts[2]), power=float(parts[3]),
+                                     hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        loaded = [r for r in rows if r["power"] > 250.0] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+                "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(loaded)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (reported baseline; test infrastructure, timed as it stands)
+# ---------------------------------------------------------------------------
+def oracle_step(P, wl, rows):
+    import oracle
+    Xq, xs = oracle.quant_act(wl.X[rows], P.s)
+    ad = wk.row_adapter(wl.seg_offsets, wl.seg_adapter, wl.M, len(wl.adapters))
+    # the sampled tokens keep their own adapters: one segment per token
+    so = np.arange(len(rows) + 1, dtype=np.int32)
+    sa = ad[rows].astype(np.int32)
+    oracle.linear_lora_rows(Xq, xs, P.Wq, P.w_scale, P.A_s, P.B_s, so, sa, want=("Y",))
+
+
+def cpu_baseline(wl, sample_rows=None):
+    import oracle
+    P = oracle.Prepared(wl)
+    rows = np.arange(wl.M if sample_rows is None else min(sample_rows, wl.M))
+    t0 = time.perf_counter()
+    oracle_step(P, wl, rows)
+    dt = time.perf_counter() - t0
+    ops = 2 * len(rows) * wl.N * wl.K
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{len(rows)} of {wl.M} tokens, whole hot path (quantize, int64 GEMM, fp64 "
+                      f"dequant + LoRA), one pass, {dt:.2f} s",
+            "tokens_per_s": len(rows) / dt}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    wl = wk.make_workload(args.workload)
+    P = oracle.Prepared(wl)
+    sample = min(wl.M, 256)
+    rng = np.random.default_rng(0)
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(wl.M, size=sample, replace=False))
+        t0 = time.perf_counter()
+        oracle_step(P, wl, rows)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    t = sum(times)
+    ops = 2 * sample * wl.N * wl.K * len(times)
+    value = ops / t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
+        "data": "synthetic",
+        "config": {"workload": wl.spec.name, "M": wl.M, "K": wl.K, "N": wl.N,
+                   "sample_tokens_per_step": sample},
+        "tokens_per_s": sample * len(times) / t,
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{sample} random tokens of {wl.M} per step, whole hot path"},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU path
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import w8a8_smoothquant_int8_b200 as sq
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    if sq.sq_device_supported(local_rank) != 0:
+        raise SystemExit("device is not compute capability 10.0")
+
+    # cpu baseline first (rank 0, N=1 only), before any CUDA work in this process
+    wl = wk.make_workload(args.workload)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl)
+
+    M, K, N = wl.M, wl.K, wl.N
+
+    def h2d(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        if a.dtype == np.uint16:
+            t = t.view(torch.bfloat16)
+        return t.to(dev)
+
+    # offline preparation (not timed): calibration, smoothing, weight quant, LoRA pack
+    X = h2d(wl.X)
+    W = h2d(wl.W)
+    act_absmax = torch.zeros(K, dtype=torch.float32, device=dev)
+    sq.sq_act_absmax_update(h2d(wl.X_cal), act_absmax)
+    w_absmax = torch.empty(K, dtype=torch.float32, device=dev)
+    sq.sq_weight_absmax(W, w_absmax)
+    s = torch.empty(K, dtype=torch.float32, device=dev)
+    sq.sq_compute_smoothing(act_absmax, w_absmax, wl.alpha, s)
+    Wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+    w_scale = torch.empty(N, dtype=torch.float32, device=dev)
+    sq.sq_quantize_weight(W, s, Wq, w_scale)
+    del W
+    lora = sq.LoraPack.build([h2d(a.A) for a in wl.adapters], [h2d(a.B) for a in wl.adapters],
+                             [a.lora_alpha for a in wl.adapters], s)
+    seg_offsets = h2d(wl.seg_offsets)
+    seg_adapter = h2d(wl.seg_adapter)
+    Xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    x_scale = torch.empty(M, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(sq.sq_linear_lora_workspace_size(M, lora.R), 256), dtype=torch.uint8,
+                     device=dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def step():
+        sq.sq_quant_act(X, s, Xq, x_scale)
+        sq.sq_linear_lora(Xq, x_scale, Wq, w_scale, lora, seg_offsets, seg_adapter, Y, ws)
+
+    launches_per_step = 3  # quantize, LoRA shrink, fused GEMM
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    n = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+    for e in ev:  # create the event handles before the library records them
+        for x in e:
+            x.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(n):
+        flush.fill_(i & 0x7f)
+        ev[i][0].record()
+        sq.sq_set_gemm_events(ev[i][2], ev[i][3])
+        step()
+        ev[i][1].record()
+    sq.sq_set_gemm_events(None, None)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    step_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    gemm_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    t_local = torch.tensor([sum(step_ms), sum(gemm_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
+    t_step_total, t_gemm_total = [float(x) for x in t_local.cpu()]
+    err = sq.sq_get_device_error(clear=True)
+    if err:
+        raise SystemExit(f"device error {err}: {sq.sq_status_string(err)}")
+
+    # end to end through the public API with host buffers: pinned X in, Y out
+    X_host = torch.from_numpy(np.ascontiguousarray(wl.X)).view(torch.bfloat16) \
+        if wl.x_is_bf16 else torch.from_numpy(np.ascontiguousarray(wl.X))
+    X_host = X_host.pin_memory()
+    Y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    e2e_ms = []
+    for i in range((args.warmup + args.e2e_steps) if args.e2e_steps > 0 else 0):
+        flush.fill_(3)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        X.copy_(X_host, non_blocking=True)
+        step()
+        Y_host.copy_(Y, non_blocking=True)
+        b.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    t_e2e = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
+    t_e2e = float(t_e2e.item())
+    e2e = None
+    if e2e_ms:
+        e2e = {"value": 2 * M * N * K * len(e2e_ms) * world / (t_e2e * 1e-3) / 1e12, "unit": "TOPS",
+               "h2d_bytes_per_step": int(X_host.numel() * X_host.element_size()),
+               "d2h_bytes_per_step": int(Y_host.numel() * Y_host.element_size()),
+               "ms_per_step": t_e2e / len(e2e_ms)}
+
+    ops_step = 2 * M * N * K
+    value = ops_step * n * world / (t_step_total * 1e-3) / 1e12
+    tok_s = M * n * world / (t_step_total * 1e-3)
+    gemm_avg_s = t_gemm_total * 1e-3 / n
+    gemm_tops = ops_step / gemm_avg_s / 1e12
+    peaks, peak_kind = measured_peaks()
+    int8_peak = 2.0 * float(peaks["bf16_tflops"])  # dense int8 = 2x dense bf16 (nominal ratio)
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TOPS",
+        "n_gpus": world,
+        "steps": n,
+        "warmup": args.warmup,
+        "ms_per_step": t_step_total / n,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8",
+        "data": "synthetic",
+        "config": {"workload": wl.spec.name, "M": M, "K": K, "N": N,
+                   "adapters": len(wl.adapters), "ranks": sorted(set(a.r for a in wl.adapters)),
+                   "segments": int(len(wl.seg_adapter)), "alpha": wl.alpha,
+                   "step": "sq_quant_act + sq_linear_lora (shrink + fused GEMM)",
+                   "l2": "flushed between timed steps (256 MiB write, untimed)",
+                   "parallelism": f"replicas x{world}"},
+        "tokens_per_s": tok_s,
+        "lora_flops_per_step": lora_flops(wl),
+        "roofline": {"bound": "tensor", "kernel": "w8a8_lora_gemm_kernel", "achieved": gemm_tops,
+                     "peak": int8_peak, "unit": "TOPS", "frac": gemm_tops / int8_peak,
+                     "peak_source": f"{peak_kind}: 2 x bf16 burst {peaks['bf16_tflops']} TFLOP/s",
+                     "gemm_us": gemm_avg_s * 1e6, "traffic": None,
+                     "algorithmic_ops": ops_step},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clocks,
+        "gpu_launches": launches_per_step * n * world,
+    }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -86,6 +86,12 @@ int sq_get_device_error(int *code, int clear);
  * SQ_ERR_DEVICE_TIMEOUT and return.  Host-side setting for later launches. */
 int sq_set_wait_timeout_ns(uint64_t ns);
 
+/* Measurement aid: when both are non-NULL, sq_linear_lora records the
+ * cudaEvent_t `before` on its stream right before it launches the fused GEMM
+ * kernel and `after` right after, so a caller can time that kernel alone.
+ * NULL disables.  Host-side setting for later calls. */
+int sq_set_gemm_events(void *before, void *after);
+
 /* ---------------------------------------------------------------------------
  * Offline preparation ("SmoothQuant" explainer, Steps 3-5 and the sketch)
  * ------------------------------------------------------------------------ */

@@ -19,7 +19,7 @@ from . import _native
 
 __all__ = [
     "SQError", "LoraPack", "sq_status_string", "sq_version", "sq_device_supported",
-    "sq_get_device_error", "sq_set_wait_timeout_ns", "sq_act_absmax_update", "sq_weight_absmax",
+    "sq_get_device_error", "sq_set_wait_timeout_ns", "sq_set_gemm_events", "sq_act_absmax_update", "sq_weight_absmax",
     "sq_compute_smoothing", "sq_quantize_weight", "sq_prepare_lora", "sq_quant_act",
     "sq_linear_lora_workspace_size", "sq_linear_lora", "sq_gemm_i32", "sq_lora_delta",
 ]
@@ -90,6 +90,13 @@ def sq_get_device_error(clear: bool = True) -> int:
 
 def sq_set_wait_timeout_ns(ns: int) -> None:
     _check(_lib().sq_set_wait_timeout_ns(int(ns)), "sq_set_wait_timeout_ns")
+
+
+def sq_set_gemm_events(before=None, after=None) -> None:
+    """Record torch.cuda.Event objects around the fused GEMM launch (None: off)."""
+    b = None if before is None else before.cuda_event
+    a = None if after is None else after.cuda_event
+    _check(_lib().sq_set_gemm_events(b, a), "sq_set_gemm_events")
 
 
 def sq_act_absmax_update(X, act_absmax, stream=None) -> None:

@@ -8,6 +8,7 @@
 namespace sq {
 
 static uint64_t g_wait_timeout_ns = 2000000000ull;
+static cudaEvent_t g_gemm_ev_before = nullptr, g_gemm_ev_after = nullptr;
 uint64_t wait_timeout_ns() { return g_wait_timeout_ns; }
 
 // ---------------------------------------------------------------------------
@@ -16,10 +17,19 @@ uint64_t wait_timeout_ns() { return g_wait_timeout_ns; }
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 static bool ptr_ok(const void *p) { return p != nullptr && aligned16(p); }
 
+// Result of sq_device_supported per device, cached: querying the device
+// properties takes far longer than a launch.
 static int check_device() {
+  static int cached[64] = {0};  // 0 = unknown, else status + 1
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SQ_ERR_CUDA;
-  return sq_device_supported(dev);
+  if (dev < 0 || dev >= 64) return sq_device_supported(dev);
+  if (cached[dev] == 0) {
+    int st = sq_device_supported(dev);
+    if (st == SQ_ERR_CUDA) return st;
+    cached[dev] = st + 1;
+  }
+  return cached[dev] - 1;
 }
 
 static int check_mk(int64_t M, int64_t K) {
@@ -93,9 +103,11 @@ const char *sq_status_string(int status) {
 int sq_version(void) { return 100; }
 
 int sq_device_supported(int device) {
-  cudaDeviceProp prop;
-  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return SQ_ERR_CUDA;
-  return (prop.major == 10 && prop.minor == 0) ? SQ_OK : SQ_ERR_UNSUPPORTED_DEVICE;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device) != cudaSuccess)
+    return SQ_ERR_CUDA;
+  return (major == 10 && minor == 0) ? SQ_OK : SQ_ERR_UNSUPPORTED_DEVICE;
 }
 
 int sq_get_device_error(int *code, int clear) {
@@ -114,6 +126,13 @@ int sq_get_device_error(int *code, int clear) {
 int sq_set_wait_timeout_ns(uint64_t ns) {
   if (ns == 0) return SQ_ERR_INVALID_ARG;
   g_wait_timeout_ns = ns;
+  return SQ_OK;
+}
+
+int sq_set_gemm_events(void *before, void *after) {
+  if ((before == nullptr) != (after == nullptr)) return SQ_ERR_INVALID_ARG;
+  g_gemm_ev_before = static_cast<cudaEvent_t>(before);
+  g_gemm_ev_after = static_cast<cudaEvent_t>(after);
   return SQ_OK;
 }
 
@@ -228,7 +247,12 @@ static int linear_common(const int8_t *Xq, const float *x_scale, const int8_t *W
     lo = LoraOperands{w.T_hi, w.T_lo, B_pack, w.mask, R};
     lop = &lo;
   }
-  return cuda_status(launch_w8a8_gemm(Xq, Wq, x_scale, w_scale, M, N, K, mode, out, lop, s));
+  const bool timed = (mode == 0) && g_gemm_ev_before != nullptr;
+  if (timed && cudaEventRecord(g_gemm_ev_before, s) != cudaSuccess) return SQ_ERR_CUDA;
+  cudaError_t e = launch_w8a8_gemm(Xq, Wq, x_scale, w_scale, M, N, K, mode, out, lop, s);
+  if (e != cudaSuccess) return SQ_ERR_CUDA;
+  if (timed && cudaEventRecord(g_gemm_ev_after, s) != cudaSuccess) return SQ_ERR_CUDA;
+  return SQ_OK;
 }
 
 int sq_linear_lora(const int8_t *Xq, const float *x_scale, const int8_t *Wq, const float *w_scale,

@@ -1,23 +1,32 @@
 // W8A8 GEMM with fused dequantization and multi-adapter LoRA delta, sm_100a.
 //
-// Computes, for a tile of 128 tokens x 256 output channels ("SmoothQuant"
+// Computes, for a tile of 256 tokens x 256 output channels ("SmoothQuant"
 // explainer, Step 7; "[Feature]: LoRA support for W8A8 SmoothQuant", Pitch):
 //   acc   = Xq Wq^T                       int8 x int8 -> int32, tensor cores
-//   delta = T_hi Bp^T + T_lo Bp^T         bf16 x bf16 -> fp32, tensor cores
-//   Y     = bf16(f32(acc) * x_scale_i * w_scale_n + delta)
+//   base  = f32(acc) * x_scale_i * w_scale_n
+//   Y     = bf16(base + T_hi Bp^T + T_lo Bp^T)   bf16 x bf16 -> fp32 on top
 // with T = (x_scale * Xq) A_pack^T from the shrink kernel, stored as two bf16
 // planes that are zero outside each token's adapter columns, so all adapters
-// present in a tile are handled by dense MMAs over the packed width.
+// of a tile are applied by dense MMAs over the packed LoRA width.
 //
-// Structure: persistent, one CTA per SM, 6 warps.
-//   warp 0     TMA producer: Xq/Wq k-blocks (and LoRA chunks) into a ring of
-//              shared-memory stages, 128-byte swizzled.
-//   warp 1     owns TMEM (512 columns) and issues tcgen05.mma:
-//              columns [0,256) int32 accumulator, [256,512) fp32 LoRA delta.
-//   warps 2-5  epilogue: tcgen05.ld -> dequant + delta -> bf16 -> global.
-// Every wait is bounded (see mbar_wait); a wait that runs out makes all roles
-// stop, drain the copies and MMAs already issued, free TMEM and record
-// SQ_ERR_DEVICE_TIMEOUT.
+// Structure: a pair of CTAs (a cluster of two, one per SM) shares each
+// 256x256 tile through tcgen05.mma.cta_group::2: each CTA stages 128 token
+// rows of Xq and 128 output-channel rows of Wq per K block, and each keeps the
+// accumulator of its 128 token rows in its own tensor memory.  Persistent:
+// one pair per two SMs walks the tiles.  Per CTA, 6 warps:
+//   warp 0     TMA producer: Xq/Wq K blocks and LoRA chunks into a ring of
+//              128-byte-swizzled shared-memory stages.  Completion of both
+//              CTAs' copies is counted on the first CTA's barrier.
+//   warp 1     allocates TMEM (two 256-column accumulator buffers); in the
+//              first CTA of the pair its lane 0 issues every MMA of the pair.
+//   warps 2-5  epilogue.  A tile with LoRA rows is finished in two passes:
+//              int32 -> base (fp32) rewritten in place in TMEM, then, after
+//              the LoRA MMAs have accumulated onto it, fp32 -> bf16 -> global.
+// The LoRA MMAs of tile i are issued a few K blocks into tile i+1, while the
+// epilogue converts tile i, so the tensor pipe does not wait for it.
+// Every wait is bounded (mbar_wait); when one runs out, all roles stop,
+// record SQ_ERR_DEVICE_TIMEOUT, wait for their own copies and MMAs, free
+// TMEM and return.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -26,18 +35,19 @@
 
 namespace sq {
 
-constexpr int BM = 128;              // tokens per tile (MMA M)
-constexpr int BN = 256;              // output channels per tile (MMA N)
+constexpr int BM = 256;              // tokens per tile (pair MMA M; 128 per CTA)
+constexpr int BN = 256;              // output channels per tile (MMA N; 128 staged per CTA)
 constexpr int BK = 128;              // int8 K elements per stage (128 bytes)
-constexpr int kStages = 4;
-constexpr int kABytes = BM * BK;     // 16 KB
-constexpr int kBBytes = BN * BK;     // 32 KB
+constexpr int kHalf = 128;           // rows each CTA stages / owns
+constexpr int kStages = 6;
+constexpr int kABytes = kHalf * BK;  // 16 KB
+constexpr int kBBytes = kHalf * BK;  // 16 KB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kLoraChunk = 64;       // bf16 columns of the LoRA width per stage
+constexpr int kDefer = 4;            // K blocks of the next tile before a tile's LoRA MMAs
 constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemAcc = 0;
-constexpr uint32_t kTmemLora = 256;
+constexpr int kEpiThreads = 128;
+constexpr uint32_t kTmemCols = 512;  // two 256-column accumulator buffers
 // Bound of the final waits for this CTA's own copies and MMAs, independent of
 // the (possibly tiny) user wait bound: those always complete.
 constexpr uint64_t kDrainNs = 1000000000ull;
@@ -50,16 +60,18 @@ struct GemmArgs {
   const float *x_scale;
   const float *w_scale;
   void *out;
-  const unsigned long long *lora_mask;  // [num_mb] 16-column group masks, or null
-  int num_mb, num_nb, num_tiles, group_m;
+  const unsigned long long *lora_mask;  // [ceil(M/128)] 16-column group masks, or null
+  int num_mb, num_nb, num_tiles, group_m, num_pairs;
   uint64_t timeout_ns;
 };
 
 struct SharedCtl {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  uint64_t acc_full;
-  uint64_t acc_empty;
+  uint64_t full[kStages];    // first CTA: both CTAs' copies of a stage landed
+  uint64_t empty[kStages];   // each CTA: the MMAs reading a stage finished
+  uint64_t acc_full[2];      // each CTA: the int8 MMAs of a buffer finished
+  uint64_t acc_empty[2];     // first CTA: both epilogues released a buffer
+  uint64_t base_ready[2];    // first CTA: both epilogues rewrote a buffer as fp32
+  uint64_t lora_done[2];     // each CTA: the LoRA MMAs of a buffer finished
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -69,7 +81,7 @@ constexpr size_t kSmemBytes = static_cast<size_t>(kStages) * kStageBytes + sizeo
 
 __device__ __forceinline__ void tile_coords(int tile, const GemmArgs &a, int &mb, int &nb) {
   // groups of group_m token tiles walk the output-channel tiles together, so
-  // the CTAs running at the same time share Xq rows and Wq columns in L2
+  // the pairs running at the same time share Xq rows and Wq columns in L2
   const int per_group = a.group_m * a.num_nb;
   const int g = tile / per_group;
   const int first = g * a.group_m;
@@ -79,12 +91,64 @@ __device__ __forceinline__ void tile_coords(int tile, const GemmArgs &a, int &mb
   nb = local / gm;
 }
 
+__device__ __forceinline__ unsigned long long tile_lora_mask(const GemmArgs &a, int mb) {
+  if (a.lora_mask == nullptr || a.mode == kEpiAcc) return 0ull;
+  const int h0 = 2 * mb, h1 = 2 * mb + 1;  // the two 128-token halves
+  const int nh = static_cast<int>((a.M + 127) / 128);
+  unsigned long long m = a.lora_mask[h0];
+  if (h1 < nh) m |= a.lora_mask[h1];
+  return m;
+}
+
 __device__ __forceinline__ void signal_abort(SharedCtl *ctl) {
   *reinterpret_cast<volatile int *>(&ctl->abort) = 1;
   record_device_error(SQ_ERR_DEVICE_TIMEOUT);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// The sequence of ring stages a pair consumes, identical for both producers
+// and the MMA issuer:  for tile i = 0, 1, ...:
+//   MAIN(i, kb) for kb < min(kDefer, nk);  LORA(i-1) chunks;  MAIN(i, kb) for
+//   kb >= kDefer;  and LORA(last) at the end.  LORA(t) = for every 64-column
+// chunk of the LoRA width the tile uses, a T_hi stage and a T_lo stage.
+// `f(kind, i, tile, a, b, first, last)` returns false to stop the walk.
+enum ItemKind : int { kMain = 0, kLora = 1, kNoMain = 2 };
+
+template <class F>
+__device__ __forceinline__ bool walk_items(const GemmArgs &args, int pair, int nk, F &&f) {
+  int i = 0, prev_tile = -1;
+  auto lora_items = [&](int ti, int tile) -> bool {
+    int mb, nb;
+    tile_coords(tile, args, mb, nb);
+    const unsigned long long mask = tile_lora_mask(args, mb);
+    if (mask == 0ull) return true;
+    int last_c = 0;
+    for (int c = 0; c < SQ_MAX_LORA_COLS / kLoraChunk; ++c)
+      if ((mask >> (4 * c)) & 0xFull) last_c = c;
+    bool first = true;
+    for (int c = 0; c < SQ_MAX_LORA_COLS / kLoraChunk; ++c) {
+      if (((mask >> (4 * c)) & 0xFull) == 0) continue;
+      for (int part = 0; part < 2; ++part) {
+        if (!f(kLora, ti, tile, c, part, first, c == last_c && part == 1)) return false;
+        first = false;
+      }
+    }
+    return true;
+  };
+  for (int tile = pair; tile < args.num_tiles; tile += args.num_pairs, ++i) {
+    const int split = min(kDefer, nk);
+    if (nk == 0 && !f(kNoMain, i, tile, 0, 0, true, true)) return false;
+    for (int kb = 0; kb < split; ++kb)
+      if (!f(kMain, i, tile, kb, 0, kb == 0, kb == nk - 1)) return false;
+    if (prev_tile >= 0 && !lora_items(i - 1, prev_tile)) return false;
+    for (int kb = split; kb < nk; ++kb)
+      if (!f(kMain, i, tile, kb, 0, kb == 0, kb == nk - 1)) return false;
+    prev_tile = tile;
+  }
+  if (prev_tile >= 0 && !lora_items(i - 1, prev_tile)) return false;
+  return true;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     w8a8_lora_gemm_kernel(const __grid_constant__ CUtensorMap tm_xq,
                           const __grid_constant__ CUtensorMap tm_wq,
                           const __grid_constant__ CUtensorMap tm_thi,
@@ -97,7 +161,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int *abort_flag = &ctl->abort;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const bool use_lora = args.lora_mask != nullptr;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs of the pair
+  const int pair = blockIdx.x >> 1;
+  const bool use_lora = args.lora_mask != nullptr && args.mode != kEpiAcc;
   // the LoRA-only epilogue needs no int8 contraction
   const int nk = (args.mode == kEpiDelta) ? 0 : static_cast<int>((args.K + BK - 1) / BK);
 
@@ -106,8 +172,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctl->full[s], 1);
       mbar_init(&ctl->empty[s], 1);
     }
-    mbar_init(&ctl->acc_full, 1);
-    mbar_init(&ctl->acc_empty, 4 * 32);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl->acc_full[b], 1);
+      mbar_init(&ctl->acc_empty[b], 2 * kEpiThreads);
+      mbar_init(&ctl->base_ready[b], 2 * kEpiThreads);
+      mbar_init(&ctl->lora_done[b], 1);
+    }
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
     fence_mbar_init();
@@ -122,11 +192,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(&ctl->tmem_base, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(&ctl->tmem_base, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive or copy
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
 
@@ -135,96 +206,89 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued = 0, issued_parity = 0;  // per-stage bit sets
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
+      const int row_off = static_cast<int>(rank) * kHalf;
+      bool ok = walk_items(args, pair, nk, [&](int kind, int, int tile, int a, int part, bool,
+                                               bool) -> bool {
+        if (kind == kNoMain) return true;
+        if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, args.timeout_ns, abort_flag)) return false;
         int mb, nb;
         tile_coords(tile, args, mb, nb);
-        const unsigned long long mask = use_lora ? args.lora_mask[mb] : 0ull;
-        for (int c = 0; ok && c < SQ_MAX_LORA_COLS / kLoraChunk; ++c) {
-          if (((mask >> (4 * c)) & 0xFull) == 0) continue;
-          for (int part = 0; part < 2; ++part) {
-            if (!(ok = mbar_wait(&ctl->empty[stage], phase ^ 1u, args.timeout_ns, abort_flag)))
-              break;
-            uint8_t *a_dst = smem + stage * kStageBytes;
-            mbar_arrive_expect_tx(&ctl->full[stage], kStageBytes);
-            tma_load_2d(a_dst, part ? &tm_tlo : &tm_thi, &ctl->full[stage], c * kLoraChunk,
-                        mb * BM);
-            tma_load_2d(a_dst + kABytes, &tm_bp, &ctl->full[stage], c * kLoraChunk, nb * BN);
-            issued |= 1u << stage;
-            issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-            if (++stage == kStages) { stage = 0; phase ^= 1u; }
-          }
+        uint8_t *a_dst = smem + stage * kStageBytes;
+        uint64_t *full_local = &ctl->full[stage];
+        const uint32_t full_pair = map_to_rank(smem_u32(full_local), 0);
+        if (rank == 0) mbar_arrive_expect_tx(full_local, 2 * kStageBytes);
+        if (kind == kMain) {
+          tma_load_2d_pair(a_dst, &tm_xq, full_pair, a * BK, mb * BM + row_off);
+          tma_load_2d_pair(a_dst + kABytes, &tm_wq, full_pair, a * BK, nb * BN + row_off);
+        } else {
+          tma_load_2d_pair(a_dst, part ? &tm_tlo : &tm_thi, full_pair, a * kLoraChunk,
+                           mb * BM + row_off);
+          tma_load_2d_pair(a_dst + kABytes, &tm_bp, full_pair, a * kLoraChunk, nb * BN + row_off);
         }
-        for (int kb = 0; ok && kb < nk; ++kb) {
-          if (!(ok = mbar_wait(&ctl->empty[stage], phase ^ 1u, args.timeout_ns, abort_flag)))
-            break;
-          uint8_t *a_dst = smem + stage * kStageBytes;
-          mbar_arrive_expect_tx(&ctl->full[stage], kStageBytes);
-          tma_load_2d(a_dst, &tm_xq, &ctl->full[stage], kb * BK, mb * BM);
-          tma_load_2d(a_dst + kABytes, &tm_wq, &ctl->full[stage], kb * BK, nb * BN);
-          issued |= 1u << stage;
-          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == kStages) { stage = 0; phase ^= 1u; }
-        }
-      }
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        return true;
+      });
       if (!ok) signal_abort(ctl);
-      // every issued copy must land before the CTA exits
-      volatile int never = 0;
-      for (int s = 0; s < kStages; ++s)
-        if (issued & (1u << s))
-          mbar_wait(&ctl->full[s], (issued_parity >> s) & 1u, kDrainNs, &never);
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
-    if (lane == 0) {
+    if (rank == 0 && lane == 0) {
       const uint32_t idesc8 = idesc_i8_s32(BM, BN);
       const uint32_t idesc16 = idesc_bf16_f32(BM, BN);
       int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
-        int mb, nb;
-        tile_coords(tile, args, mb, nb);
-        const unsigned long long mask = use_lora ? args.lora_mask[mb] : 0ull;
-        if (!(ok = mbar_wait(&ctl->acc_empty, acc_phase ^ 1u, args.timeout_ns, abort_flag))) break;
-        tc_fence_after();
-        uint32_t lora_acc = 0;
-        for (int c = 0; ok && c < SQ_MAX_LORA_COLS / kLoraChunk; ++c) {
-          const unsigned groups = static_cast<unsigned>((mask >> (4 * c)) & 0xFull);
-          if (groups == 0) continue;
-          for (int part = 0; part < 2; ++part) {
-            if (!(ok = mbar_wait(&ctl->full[stage], phase, args.timeout_ns, abort_flag))) break;
-            tc_fence_after();
-            const uint32_t a_base = smem_u32(smem + stage * kStageBytes);
-            const uint32_t b_base = a_base + kABytes;
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              if (groups & (1u << g)) {
-                mma_f16(tmem + kTmemLora, sdesc_kmajor_sw128(a_base + 32 * g),
-                        sdesc_kmajor_sw128(b_base + 32 * g), idesc16, lora_acc);
-                lora_acc = 1;
-              }
-            }
-            mma_commit(&ctl->empty[stage]);
-            if (++stage == kStages) { stage = 0; phase ^= 1u; }
-          }
-        }
-        for (int kb = 0; ok && kb < nk; ++kb) {
-          if (!(ok = mbar_wait(&ctl->full[stage], phase, args.timeout_ns, abort_flag))) break;
+      uint32_t phase = 0;
+      uint32_t lora_uses[2] = {0, 0};
+      bool ok = walk_items(args, pair, nk, [&](int kind, int i, int tile, int a, int, bool first,
+                                               bool last) -> bool {
+        const int b = i & 1;
+        const uint32_t dbuf = tmem + static_cast<uint32_t>(b) * 256u;
+        if (kind != kLora && first) {
+          // the buffer is free once both epilogues finished tile i-2
+          if (!mbar_wait_cluster(&ctl->acc_empty[b], ((i >> 1) & 1) ^ 1u, args.timeout_ns,
+                                 abort_flag))
+            return false;
           tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + stage * kStageBytes);
-          const uint32_t b_base = a_base + kABytes;
+        }
+        if (kind == kNoMain) {
+          mma_commit_pair(&ctl->acc_full[b], 0x3);
+          return true;
+        }
+        if (kind == kLora && first) {
+          // the epilogues have rewritten the accumulator as fp32 base values
+          if (!mbar_wait_cluster(&ctl->base_ready[b], lora_uses[b] & 1u, args.timeout_ns,
+                                 abort_flag))
+            return false;
+          tc_fence_after();
+        }
+        if (!mbar_wait(&ctl->full[stage], phase, args.timeout_ns, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(smem + stage * kStageBytes);
+        const uint32_t b_base = a_base + kABytes;
+        if (kind == kMain) {
 #pragma unroll
           for (int j = 0; j < BK / 32; ++j)
-            mma_i8(tmem + kTmemAcc, sdesc_kmajor_sw128(a_base + 32 * j),
-                   sdesc_kmajor_sw128(b_base + 32 * j), idesc8, (kb | j) ? 1u : 0u);
-          mma_commit(&ctl->empty[stage]);
-          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+            mma_i8_pair(dbuf, sdesc_kmajor_sw128(a_base + 32 * j),
+                        sdesc_kmajor_sw128(b_base + 32 * j), idesc8, (a | j) ? 1u : 0u);
+        } else {
+          int mb, nb;
+          tile_coords(tile, args, mb, nb);
+          const unsigned groups =
+              static_cast<unsigned>((tile_lora_mask(args, mb) >> (4 * a)) & 0xFull);
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            if (groups & (1u << g))
+              mma_f16_pair(dbuf, sdesc_kmajor_sw128(a_base + 32 * g),
+                           sdesc_kmajor_sw128(b_base + 32 * g), idesc16, 1u);
         }
-        if (ok) mma_commit(&ctl->acc_full);
-        acc_phase ^= 1u;
-      }
+        mma_commit_pair(&ctl->empty[stage], 0x3);
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        if (kind == kMain && last) mma_commit_pair(&ctl->acc_full[b], 0x3);
+        if (kind == kLora && last) {
+          mma_commit_pair(&ctl->lora_done[b], 0x3);
+          ++lora_uses[b];
+        }
+        return true;
+      });
       if (!ok) signal_abort(ctl);
       // all MMAs issued by this thread must finish before TMEM is freed
       mma_commit(&ctl->drain);
@@ -234,42 +298,79 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter+32)
-    const int row_in_tile = quarter * 32 + lane;
+    const int row_in_tile = static_cast<int>(rank) * kHalf + quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    uint32_t acc_phase = 0;
+    const uint32_t acc_empty_pair = map_to_rank(smem_u32(&ctl->acc_empty[0]), 0);
+    const uint32_t base_ready_pair = map_to_rank(smem_u32(&ctl->base_ready[0]), 0);
+    uint32_t lora_uses[2] = {0, 0};
     bool ok = true;
-    for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x) {
+    int i = 0;
+    for (int tile = pair; tile < args.num_tiles; tile += args.num_pairs, ++i) {
+      const int b = i & 1;
+      const uint32_t dbuf = tmem + static_cast<uint32_t>(b) * 256u + lane_addr;
       int mb, nb;
       tile_coords(tile, args, mb, nb);
-      const bool has_lora = use_lora && args.lora_mask[mb] != 0ull;
-      if (!(ok = mbar_wait(&ctl->acc_full, acc_phase, args.timeout_ns, abort_flag))) break;
+      const bool has_lora = use_lora && tile_lora_mask(args, mb) != 0ull;
+      if (!(ok = mbar_wait(&ctl->acc_full[b], (i >> 1) & 1, args.timeout_ns, abort_flag))) break;
       tc_fence_after();
       const int64_t row = static_cast<int64_t>(mb) * BM + row_in_tile;
       const bool row_ok = row < args.M;
       const float xs = (row_ok && args.mode == kEpiY) ? args.x_scale[row] : 0.f;
+      if (has_lora) {
+        // pass 1: base values rewritten in place as fp32
+        for (int c = 0; c < BN / 32; ++c) {
+          const int64_t col0 = static_cast<int64_t>(nb) * BN + c * 32;
+          uint32_t v[32];
+          if (args.mode == kEpiY) {
+            tmem_ld_32x32b_x32(dbuf + c * 32, v);
+            tmem_ld_wait();
+            const float *ws = args.w_scale + col0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float w = (col0 + j < args.N) ? __ldg(ws + j) : 0.f;
+              v[j] = __float_as_uint(
+                  __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j])), xs), w));
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0u;
+          }
+          tmem_st_32x32b_x32(dbuf + c * 32, v);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive_cluster(base_ready_pair + 8u * b);
+        if (!(ok = mbar_wait(&ctl->lora_done[b], lora_uses[b] & 1u, args.timeout_ns, abort_flag)))
+          break;
+        ++lora_uses[b];
+        tc_fence_after();
+      }
+      // final pass: TMEM -> global
       for (int c = 0; c < BN / 32; ++c) {
         const int64_t col0 = static_cast<int64_t>(nb) * BN + c * 32;
         if (col0 >= args.N) break;
         const int nvalid = (col0 + 32 <= args.N) ? 32 : static_cast<int>(args.N - col0);
-        uint32_t acc[32], dl[32];
-        if (args.mode != kEpiDelta) tmem_ld_32x32b_x32(tmem + kTmemAcc + lane_addr + c * 32, acc);
-        if (has_lora) tmem_ld_32x32b_x32(tmem + kTmemLora + lane_addr + c * 32, dl);
-        tmem_ld_wait();
+        uint32_t v[32];
+        const bool zero = (args.mode == kEpiDelta) && !has_lora;
+        if (!zero) {
+          tmem_ld_32x32b_x32(dbuf + c * 32, v);
+          tmem_ld_wait();
+        }
         if (!row_ok) continue;
         if (args.mode == kEpiY) {
-          const float *ws = args.w_scale + col0;
           uint32_t packed[16];
+          const float *ws = args.w_scale + col0;
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            float v0 = 0.f, v1 = 0.f;
-            if (j < nvalid) {
-              v0 = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(acc[j])), xs), __ldg(ws + j));
-              v1 = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(acc[j + 1])), xs),
-                             __ldg(ws + j + 1));
-              if (has_lora) {
-                v0 = __fadd_rn(v0, __uint_as_float(dl[j]));
-                v1 = __fadd_rn(v1, __uint_as_float(dl[j + 1]));
-              }
+            float v0, v1;
+            if (has_lora) {
+              v0 = __uint_as_float(v[j]);
+              v1 = __uint_as_float(v[j + 1]);
+            } else {
+              const float w0 = (j < nvalid) ? __ldg(ws + j) : 0.f;
+              const float w1 = (j + 1 < nvalid) ? __ldg(ws + j + 1) : 0.f;
+              v0 = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j])), xs), w0);
+              v1 = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j + 1])), xs), w1);
             }
             __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
             packed[j / 2] = *reinterpret_cast<uint32_t *>(&h);
@@ -279,32 +380,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int t = 0; t < 4; ++t)
             if (t * 8 < nvalid)
               dst[t] = make_uint4(packed[4 * t], packed[4 * t + 1], packed[4 * t + 2], packed[4 * t + 3]);
-        } else if (args.mode == kEpiAcc) {
-          uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint32_t *>(args.out) + row * args.N + col0);
-#pragma unroll
-          for (int t = 0; t < 8; ++t)
-            if (t * 4 < nvalid)
-              dst[t] = make_uint4(acc[4 * t], acc[4 * t + 1], acc[4 * t + 2], acc[4 * t + 3]);
         } else {
           uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint32_t *>(args.out) + row * args.N + col0);
 #pragma unroll
           for (int t = 0; t < 8; ++t)
             if (t * 4 < nvalid)
-              dst[t] = has_lora ? make_uint4(dl[4 * t], dl[4 * t + 1], dl[4 * t + 2], dl[4 * t + 3])
-                                : make_uint4(0, 0, 0, 0);
+              dst[t] = zero ? make_uint4(0, 0, 0, 0)
+                            : make_uint4(v[4 * t], v[4 * t + 1], v[4 * t + 2], v[4 * t + 3]);
         }
       }
       tc_fence_before();
-      mbar_arrive(&ctl->acc_empty);
-      acc_phase ^= 1u;
+      mbar_arrive_cluster(acc_empty_pair + 8u * b);
     }
     if (!ok) signal_abort(ctl);
   }
 
+  if (*abort_flag) {
+    // a stopped pair may still have copies in flight: give them time to land
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 100000ull) {
+    }
+  }
+  tc_fence_before();
   __syncthreads();
+  cluster_sync();  // neither CTA leaves while its peer may still touch it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc_pair(tmem, kTmemCols);
   }
 }
 
@@ -365,11 +467,11 @@ cudaError_t launch_w8a8_gemm(const int8_t *Xq, const int8_t *Wq, const float *x_
   memset(&tm_thi, 0, sizeof tm_thi);
   memset(&tm_tlo, 0, sizeof tm_tlo);
   memset(&tm_bp, 0, sizeof tm_bp);
-  if (!make_tmap(&tm_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, BK, BM))
+  if (!make_tmap(&tm_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, BK, kHalf))
     return cudaErrorInvalidValue;
   if (mode == kEpiDelta)
     tm_wq = tm_xq;  // never loaded: the LoRA-only epilogue skips the int8 mainloop
-  else if (!make_tmap(&tm_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, BK, BN))
+  else if (!make_tmap(&tm_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, BK, kHalf))
     return cudaErrorInvalidValue;
   GemmArgs a;
   a.M = M;
@@ -380,20 +482,21 @@ cudaError_t launch_w8a8_gemm(const int8_t *Xq, const int8_t *Wq, const float *x_
   a.w_scale = w_scale;
   a.out = out;
   a.lora_mask = nullptr;
-  if (lora && lora->R > 0) {
+  if (lora && lora->R > 0 && mode != kEpiAcc) {
     if (!make_tmap(&tm_thi, lora->T_hi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lora->R, M,
-                   kLoraChunk, BM) ||
+                   kLoraChunk, kHalf) ||
         !make_tmap(&tm_tlo, lora->T_lo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lora->R, M,
-                   kLoraChunk, BM) ||
+                   kLoraChunk, kHalf) ||
         !make_tmap(&tm_bp, lora->B_pack, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lora->R, N,
-                   kLoraChunk, BN))
+                   kLoraChunk, kHalf))
       return cudaErrorInvalidValue;
     a.lora_mask = lora->mask;
   }
   a.num_mb = static_cast<int>((M + BM - 1) / BM);
   a.num_nb = static_cast<int>((N + BN - 1) / BN);
   a.num_tiles = a.num_mb * a.num_nb;
-  a.group_m = 8;
+  a.group_m = 4;
+  a.num_pairs = min(a.num_tiles, sm_count_of_current_device() / 2);
   a.timeout_ns = wait_timeout_ns();
   static bool attr_set = false;
   if (!attr_set) {
@@ -403,8 +506,8 @@ cudaError_t launch_w8a8_gemm(const int8_t *Xq, const int8_t *Wq, const float *x_
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int grid = min(a.num_tiles, sm_count_of_current_device());
-  w8a8_lora_gemm_kernel<<<grid, kThreads, kSmemBytes, st>>>(tm_xq, tm_wq, tm_thi, tm_tlo, tm_bp, a);
+  w8a8_lora_gemm_kernel<<<2 * a.num_pairs, kThreads, kSmemBytes, st>>>(tm_xq, tm_wq, tm_thi, tm_tlo,
+                                                                       tm_bp, a);
   return cudaGetLastError();
 }
 

@@ -2,7 +2,7 @@
 //   T[i, j] = x_scale_i * sum_k Xq[i,k] * A_pack[off_a + j, k]   (j < r_a)
 // for the adapter a of token i ("[Feature]: LoRA support for W8A8
 // SmoothQuant", Pitch: the LoRA path runs after the INT8 GEMM in BF16; A_pack
-// carries the smoothing scale so Xq*x_scale*diag(s) ~ X).
+// carries the smoothing scale so that Xq*x_scale*diag(s) ~ X).
 //
 // T is written as two bf16 planes over the packed width R, T_hi = bf16(T) and
 // T_lo = bf16(T - T_hi), with zeros outside the token's adapter columns, so
@@ -10,108 +10,251 @@
 // dense bf16 tensor-core MMAs and still carry ~16 significant bits of T.
 // mask[tile] collects, per 128-token tile, the 16-column groups of R that
 // some token of the tile uses.
+//
+// The contraction is a skinny GEMM (N = rank <= 64 per pass) done with
+// warp-level bf16 tensor-core MMAs (m16n8k16, fp32 accumulation): the int8
+// codes are exact in bf16, so converting them in registers loses nothing.
+// Each thread loads 16 contiguous K-bytes of its two rows per 64-wide K chunk;
+// within a chunk the K order seen by the MMA is a permutation that both
+// operands share, which leaves the dot products unchanged.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
 
 namespace sq {
 
-constexpr int kShrinkThreads = 128;
+constexpr int kShrinkWarps = 8;
+constexpr int kShrinkThreads = 32 * kShrinkWarps;
 
+__device__ __forceinline__ uint32_t bf16x2_of_s8(uint32_t w, int first_byte) {
+  // two consecutive signed bytes -> packed bf16 pair (exact)
+  const float lo = static_cast<float>(static_cast<int8_t>((w >> (8 * first_byte)) & 0xffu));
+  const float hi = static_cast<float>(static_cast<int8_t>((w >> (8 * first_byte + 8)) & 0xffu));
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Partial products of 16 rows [row0, row0+16) with 8*kNT consecutive rows of
+// A_pack starting at `arow0`, over the 64-wide K chunks c = c_begin,
+// c_begin + c_step, ...  acc[nt][.] is the m16n8 fragment of columns
+// [8nt, 8nt+8).  Two chunks are loaded before either is used, so that each
+// warp keeps twice the bytes in flight.
+template <int kNT>
+__device__ __forceinline__ void shrink_warp_tile(const int8_t *__restrict__ Xq, int64_t M,
+                                                 int64_t K, int64_t row0,
+                                                 const uint16_t *__restrict__ A_pack, int64_t arow0,
+                                                 int c_begin, int c_step, float (&acc)[8][4]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
+  const int64_t ra = row0 + g, rb = row0 + g + 8;
+  const int nchunks = static_cast<int>((K + 63) / 64);
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int t = 0; t < 4; ++t) acc[nt][t] = 0.f;
+  constexpr int kDepth = (kNT <= 4) ? 2 : 1;
+  for (int c0 = c_begin; c0 < nchunks; c0 += kDepth * c_step) {
+    uint4 xa[kDepth], xb[kDepth], bv[kDepth][kNT][2];
+#pragma unroll
+    for (int d = 0; d < kDepth; ++d) {
+      const int c = c0 + d * c_step;
+      const int64_t k = static_cast<int64_t>(c) * 64 + 16 * tig;
+      const bool kin = c < nchunks && k < K;  // K % 16 == 0: a 16-slice is all in or out
+      xa[d] = make_uint4(0, 0, 0, 0);
+      xb[d] = make_uint4(0, 0, 0, 0);
+      if (kin && ra < M) xa[d] = __ldg(reinterpret_cast<const uint4 *>(Xq + ra * K + k));
+      if (kin && rb < M) xb[d] = __ldg(reinterpret_cast<const uint4 *>(Xq + rb * K + k));
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) {
+        bv[d][nt][0] = make_uint4(0, 0, 0, 0);
+        bv[d][nt][1] = make_uint4(0, 0, 0, 0);
+        if (kin) {
+          const uint16_t *ap = A_pack + (arow0 + nt * 8 + g) * K + k;
+          bv[d][nt][0] = __ldg(reinterpret_cast<const uint4 *>(ap));
+          bv[d][nt][1] = __ldg(reinterpret_cast<const uint4 *>(ap + 8));
+        }
+      }
+    }
+#pragma unroll
+    for (int d = 0; d < kDepth; ++d) {
+      const uint32_t wa[4] = {xa[d].x, xa[d].y, xa[d].z, xa[d].w};
+      const uint32_t wb[4] = {xb[d].x, xb[d].y, xb[d].z, xb[d].w};
+      uint32_t afrag[4][4];  // [k16 step][a0..a3]
+#pragma unroll
+      for (int st = 0; st < 4; ++st) {
+        afrag[st][0] = bf16x2_of_s8(wa[st], 0);
+        afrag[st][1] = bf16x2_of_s8(wb[st], 0);
+        afrag[st][2] = bf16x2_of_s8(wa[st], 2);
+        afrag[st][3] = bf16x2_of_s8(wb[st], 2);
+      }
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) {
+        const uint32_t bw[8] = {bv[d][nt][0].x, bv[d][nt][0].y, bv[d][nt][0].z, bv[d][nt][0].w,
+                                bv[d][nt][1].x, bv[d][nt][1].y, bv[d][nt][1].z, bv[d][nt][1].w};
+#pragma unroll
+        for (int st = 0; st < 4; ++st)
+          mma_bf16_16816(acc[nt], afrag[st], bw[2 * st], bw[2 * st + 1]);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void store_t_pair(uint16_t *T_hi, uint16_t *T_lo, int64_t idx, float v0,
+                                             float v1) {
+  __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
+  __nv_bfloat16 l0 = __float2bfloat16_rn(v0 - __bfloat162float(h0));
+  __nv_bfloat16 l1 = __float2bfloat16_rn(v1 - __bfloat162float(h1));
+  *reinterpret_cast<uint32_t *>(T_hi + idx) =
+      static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+      (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+  *reinterpret_cast<uint32_t *>(T_lo + idx) =
+      static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
+      (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+}
+
+// A block of 8 warps covers kRG groups of 16 rows; the kKS = 8/kRG warps of a
+// row group split K between them and add their partial sums in a fixed order
+// through shared memory.  More row groups per block means more reuse of the
+// adapter rows through L1; more K splits means more blocks for small M.
+__device__ __forceinline__ void group_sync(int rg, int nwarps) {
+  if (nwarps == 1)
+    __syncwarp();
+  else
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + rg), "r"(nwarps * 32) : "memory");
+}
+
+template <int kRG>
 __global__ void __launch_bounds__(kShrinkThreads) lora_shrink_kernel(
-    const int8_t *__restrict__ Xq, const float *__restrict__ x_scale, int64_t K,
+    const int8_t *__restrict__ Xq, const float *__restrict__ x_scale, int64_t M, int64_t K,
     const uint16_t *__restrict__ A_pack, const int32_t *__restrict__ lora_offset,
     const int32_t *__restrict__ lora_rank, int n_adapters, int64_t R,
     const int32_t *__restrict__ seg_offsets, const int32_t *__restrict__ seg_adapter, int64_t S,
     uint16_t *__restrict__ T_hi, uint16_t *__restrict__ T_lo,
     unsigned long long *__restrict__ mask) {
-  __shared__ float tv[SQ_MAX_LORA_COLS];
-  __shared__ float part[kShrinkThreads / 32][16];
-  __shared__ int s_off, s_rank;
-  const int64_t i = blockIdx.x;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid == 0) {
-    int a = token_adapter(seg_offsets, seg_adapter, S, n_adapters, i);
-    int off = -1, r = 0;
+  constexpr int kKS = kShrinkWarps / kRG;
+  __shared__ float red[kShrinkWarps][16][64 + 1];
+  __shared__ int s_ad[kRG][16];
+  __shared__ int s_off[kRG][16];
+  __shared__ int s_rank[kRG][16];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
+  const int rg = warp / kKS, ks = warp % kKS;
+  const int64_t row0 = (static_cast<int64_t>(blockIdx.x) * kRG + rg) * 16;
+
+  // adapter, column offset and rank of each of the 16 rows of the group
+  if (ks == 0 && lane < 16) {
+    const int64_t i = row0 + lane;
+    int a = (i < M) ? token_adapter(seg_offsets, seg_adapter, S, n_adapters, i) : -1;
+    int off = 0, r = 0;
     if (a >= 0) {
       off = lora_offset[a];
       r = lora_rank[a];
-      const int rpad = (r + 15) & ~15;
-      if (off < 0 || (off & 15) || r <= 0 || off + rpad > R) {
+      if (off < 0 || (off & 15) || r <= 0 || off + ((r + 15) & ~15) > R) {
         record_device_error(SQ_ERR_BAD_SEGMENTS);
-        off = -1;
-        r = 0;
-      } else {
-        unsigned long long bits = 0;
-        for (int g = off / 16; g < (off + rpad) / 16; ++g) bits |= 1ull << g;
-        atomicOr(mask + (i >> 7), bits);
+        a = -1;
       }
     }
-    s_off = off;
-    s_rank = r;
+    s_ad[rg][lane] = a;
+    s_off[rg][lane] = off;
+    s_rank[rg][lane] = r;
   }
   __syncthreads();
-  const int off = s_off, r = s_rank;
-  const float xs = x_scale[i];
-  const int8_t *xrow = Xq + i * K;
-  for (int g0 = 0; g0 < r; g0 += 16) {
-    float acc[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-    const int jn = min(16, r - g0);
-    for (int64_t k0 = static_cast<int64_t>(tid) * 16; k0 < K; k0 += kShrinkThreads * 16) {
-      uint4 xr = *reinterpret_cast<const uint4 *>(xrow + k0);
-      float xv[16];
-      const uint32_t w4[4] = {xr.x, xr.y, xr.z, xr.w};
-#pragma unroll
-      for (int t = 0; t < 16; ++t)
-        xv[t] = static_cast<float>(static_cast<int8_t>((w4[t >> 2] >> (8 * (t & 3))) & 0xff));
-      for (int j = 0; j < jn; ++j) {
-        const uint16_t *arow = A_pack + static_cast<int64_t>(off + g0 + j) * K + k0;
-        uint4 a0 = *reinterpret_cast<const uint4 *>(arow);
-        uint4 a1 = *reinterpret_cast<const uint4 *>(arow + 8);
-        const uint32_t av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        float s = 0.f;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          s = fmaf(xv[2 * t], __uint_as_float(av[t] << 16), s);
-          s = fmaf(xv[2 * t + 1], __uint_as_float(av[t] & 0xffff0000u), s);
-        }
-        acc[j] += s;
+  if (row0 >= M) return;  // whole row group; only group barriers follow
+
+  // zero both planes for the group's rows, and set the tile mask
+  {
+    const int64_t nrows = (M - row0 < 16) ? (M - row0) : 16;
+    const int64_t words = nrows * R / 8;  // 16-byte words (R % 16 == 0)
+    const int tid = ks * 32 + lane;
+    for (int64_t w = tid; w < words; w += kKS * 32) {
+      reinterpret_cast<uint4 *>(T_hi + row0 * R)[w] = make_uint4(0, 0, 0, 0);
+      reinterpret_cast<uint4 *>(T_lo + row0 * R)[w] = make_uint4(0, 0, 0, 0);
+    }
+    if (tid == 0) {
+      unsigned long long bits = 0;
+      for (int r = 0; r < 16; ++r) {
+        if (s_ad[rg][r] < 0) continue;
+        const int off = s_off[rg][r], rpad = (s_rank[rg][r] + 15) & ~15;
+        for (int gi = off / 16; gi < (off + rpad) / 16; ++gi) bits |= 1ull << gi;
       }
+      if (bits) atomicOr(mask + (row0 >> 7), bits);
     }
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      float v = acc[j];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) part[warp][j] = v;
-    }
-    __syncthreads();
-    if (tid < 16) {
-      float v = 0.f;
-#pragma unroll
-      for (int w = 0; w < kShrinkThreads / 32; ++w) v += part[w][tid];
-      tv[g0 + tid] = (g0 + tid < r) ? xs * v : 0.f;
-    }
-    __syncthreads();
   }
-  // write the full row of both planes: own columns from tv, zeros elsewhere
-  const int rpad = (r + 15) & ~15;
-  for (int64_t c0 = static_cast<int64_t>(tid) * 8; c0 < R; c0 += kShrinkThreads * 8) {
-    uint32_t hi[4] = {0, 0, 0, 0}, lo[4] = {0, 0, 0, 0};
-    if (off >= 0 && c0 >= off && c0 < off + rpad) {
+  group_sync(rg, kKS);
+
+  // one pass per distinct adapter among the 16 rows (usually one)
+  unsigned done = 0;  // bit r: row r handled
+  for (int r = 0; r < 16; ++r)
+    if (s_ad[rg][r] < 0) done |= 1u << r;
+  while (done != 0xffffu) {
+    const int first = __ffs(~done) - 1;
+    const int a = s_ad[rg][first], off = s_off[rg][first], rank = s_rank[rg][first];
+    unsigned rows_a = 0;
+    for (int r = 0; r < 16; ++r)
+      if (s_ad[rg][r] == a) rows_a |= 1u << r;
+    const int rpad = (rank + 15) & ~15;
+    for (int cb = 0; cb < rpad; cb += 64) {
+      const int ncols = min(64, rpad - cb);
+      float acc[8][4];
+      if (ncols <= 16)
+        shrink_warp_tile<2>(Xq, M, K, row0, A_pack, off + cb, ks, kKS, acc);
+      else if (ncols <= 32)
+        shrink_warp_tile<4>(Xq, M, K, row0, A_pack, off + cb, ks, kKS, acc);
+      else
+        shrink_warp_tile<8>(Xq, M, K, row0, A_pack, off + cb, ks, kKS, acc);
+      if (kKS > 1) {
+        // fixed-order sum of the group's K parts through shared memory
 #pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        float v = tv[c0 - off + t];
-        __nv_bfloat16 h = __float2bfloat16_rn(v);
-        __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
-        hi[t >> 1] |= static_cast<uint32_t>(__bfloat16_as_ushort(h)) << (16 * (t & 1));
-        lo[t >> 1] |= static_cast<uint32_t>(__bfloat16_as_ushort(l)) << (16 * (t & 1));
+        for (int nt = 0; nt < 8; ++nt) {
+          if (nt * 8 >= ncols) break;
+          red[warp][g][nt * 8 + 2 * tig] = acc[nt][0];
+          red[warp][g][nt * 8 + 2 * tig + 1] = acc[nt][1];
+          red[warp][g + 8][nt * 8 + 2 * tig] = acc[nt][2];
+          red[warp][g + 8][nt * 8 + 2 * tig + 1] = acc[nt][3];
+        }
+        group_sync(rg, kKS);
+        if (ks == 0) {
+#pragma unroll
+          for (int nt = 0; nt < 8; ++nt) {
+            if (nt * 8 >= ncols) break;
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const int rr = g + ((h & 2) ? 8 : 0), cc = nt * 8 + 2 * tig + (h & 1);
+              float t = red[rg * kKS][rr][cc];
+#pragma unroll
+              for (int w = 1; w < kKS; ++w) t += red[rg * kKS + w][rr][cc];
+              acc[nt][h] = t;
+            }
+          }
+        }
       }
+      if (ks == 0) {
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+          if (nt * 8 >= ncols) break;
+          const int col = cb + nt * 8 + 2 * tig;  // column within the adapter
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int rr = g + 8 * half;
+            const int64_t i = row0 + rr;
+            if (!((rows_a >> rr) & 1u) || i >= M) continue;
+            const float xs = x_scale[i];
+            const float v0 = (col < rank) ? xs * acc[nt][2 * half] : 0.f;
+            const float v1 = (col + 1 < rank) ? xs * acc[nt][2 * half + 1] : 0.f;
+            store_t_pair(T_hi, T_lo, i * R + off + col, v0, v1);
+          }
+        }
+      }
+      if (kKS > 1) group_sync(rg, kKS);
     }
-    *reinterpret_cast<uint4 *>(T_hi + i * R + c0) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    *reinterpret_cast<uint4 *>(T_lo + i * R + c0) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    done |= rows_a;
   }
 }
 
@@ -124,9 +267,25 @@ cudaError_t launch_lora_shrink(const int8_t *Xq, const float *x_scale, int64_t M
   if (M == 0) return cudaSuccess;
   cudaError_t e = cudaMemsetAsync(mask, 0, static_cast<size_t>((M + 127) / 128) * 8, st);
   if (e != cudaSuccess) return e;
-  lora_shrink_kernel<<<static_cast<unsigned>(M), kShrinkThreads, 0, st>>>(
-      Xq, x_scale, K, A_pack, lora_offset, lora_rank, n_adapters, R, seg_offsets, seg_adapter, S,
-      T_hi, T_lo, mask);
+  const int64_t row_tiles = (M + 15) / 16;
+  // widest row grouping that still leaves about two blocks per SM
+  const unsigned g1 = static_cast<unsigned>(row_tiles);
+  if (row_tiles >= 8 * 2 * 148)
+    lora_shrink_kernel<8><<<(g1 + 7) / 8, kShrinkThreads, 0, st>>>(
+        Xq, x_scale, M, K, A_pack, lora_offset, lora_rank, n_adapters, R, seg_offsets, seg_adapter,
+        S, T_hi, T_lo, mask);
+  else if (row_tiles >= 4 * 2 * 148)
+    lora_shrink_kernel<4><<<(g1 + 3) / 4, kShrinkThreads, 0, st>>>(
+        Xq, x_scale, M, K, A_pack, lora_offset, lora_rank, n_adapters, R, seg_offsets, seg_adapter,
+        S, T_hi, T_lo, mask);
+  else if (row_tiles >= 2 * 2 * 148)
+    lora_shrink_kernel<2><<<(g1 + 1) / 2, kShrinkThreads, 0, st>>>(
+        Xq, x_scale, M, K, A_pack, lora_offset, lora_rank, n_adapters, R, seg_offsets, seg_adapter,
+        S, T_hi, T_lo, mask);
+  else
+    lora_shrink_kernel<1><<<g1, kShrinkThreads, 0, st>>>(
+        Xq, x_scale, M, K, A_pack, lora_offset, lora_rank, n_adapters, R, seg_offsets, seg_adapter,
+        S, T_hi, T_lo, mask);
   return cudaGetLastError();
 }
 
