@@ -19,11 +19,12 @@
 //              CTAs' copies is counted on the first CTA's barrier.
 //   warp 1     allocates TMEM (two 256-column accumulator buffers); in the
 //              first CTA of the pair its lane 0 issues every MMA of the pair.
-//   warps 2-5  epilogue.  A tile with LoRA rows is finished in two passes:
+//   warps 2-9  epilogue (two warps per TMEM lane quarter, 128 columns each).
+//              A tile with LoRA rows is finished in two passes:
 //              int32 -> base (fp32) rewritten in place in TMEM, then, after
 //              the LoRA MMAs have accumulated onto it, fp32 -> bf16 -> global.
-// The LoRA MMAs of tile i are issued a few K blocks into tile i+1, while the
-// epilogue converts tile i, so the tensor pipe does not wait for it.
+// The LoRA MMAs of tile i are issued half way through tile i+1, after the
+// epilogue has converted tile i, so the tensor pipe does not wait for it.
 // Every wait is bounded (mbar_wait); when one runs out, all roles stop,
 // record SQ_ERR_DEVICE_TIMEOUT, wait for their own copies and MMAs, free
 // TMEM and return.
@@ -44,9 +45,9 @@ constexpr int kABytes = kHalf * BK;  // 16 KB
 constexpr int kBBytes = kHalf * BK;  // 16 KB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kLoraChunk = 64;       // bf16 columns of the LoRA width per stage
-constexpr int kDefer = 4;            // K blocks of the next tile before a tile's LoRA MMAs
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
+constexpr int kThreads = 320;        // producer warp, MMA warp, 8 epilogue warps
+constexpr int kEpiWarps = 8;         // two per TMEM lane quarter, each owning 128 columns
+constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;  // two 256-column accumulator buffers
 // Bound of the final waits for this CTA's own copies and MMAs, independent of
 // the (possibly tiny) user wait bound: those always complete.
@@ -107,8 +108,9 @@ __device__ __forceinline__ void signal_abort(SharedCtl *ctl) {
 
 // The sequence of ring stages a pair consumes, identical for both producers
 // and the MMA issuer:  for tile i = 0, 1, ...:
-//   MAIN(i, kb) for kb < min(kDefer, nk);  LORA(i-1) chunks;  MAIN(i, kb) for
-//   kb >= kDefer;  and LORA(last) at the end.  LORA(t) = for every 64-column
+//   MAIN(i, kb) for kb < split;  LORA(i-1) chunks;  MAIN(i, kb) for kb >= split;
+// and LORA(last) at the end, with split = nk/2 (the epilogue rewrites tile
+// i-1 as fp32 during the first half of tile i; the LoRA MMAs follow).  LORA(t) = for every 64-column
 // chunk of the LoRA width the tile uses, a T_hi stage and a T_lo stage.
 // `f(kind, i, tile, a, b, first, last)` returns false to stop the walk.
 enum ItemKind : int { kMain = 0, kLora = 1, kNoMain = 2 };
@@ -135,7 +137,7 @@ __device__ __forceinline__ bool walk_items(const GemmArgs &args, int pair, int n
     return true;
   };
   for (int tile = pair; tile < args.num_tiles; tile += args.num_pairs, ++i) {
-    const int split = min(kDefer, nk);
+    const int split = (nk + 1) / 2;
     if (nk == 0 && !f(kNoMain, i, tile, 0, 0, true, true)) return false;
     for (int kb = 0; kb < split; ++kb)
       if (!f(kMain, i, tile, kb, 0, kb == 0, kb == nk - 1)) return false;
@@ -297,7 +299,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter+32)
+    const int ew = warp - 2;               // epilogue warp 0..7
+    const int quarter = warp & 3;          // TMEM lanes [32*quarter, 32*quarter+32)
+    const int col_half = ew >> 2;          // columns [128*col_half, 128*col_half+128)
     const int row_in_tile = static_cast<int>(rank) * kHalf + quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t acc_empty_pair = map_to_rank(smem_u32(&ctl->acc_empty[0]), 0);
@@ -318,19 +322,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const float xs = (row_ok && args.mode == kEpiY) ? args.x_scale[row] : 0.f;
       if (has_lora) {
         // pass 1: base values rewritten in place as fp32
-        for (int c = 0; c < BN / 32; ++c) {
-          const int64_t col0 = static_cast<int64_t>(nb) * BN + c * 32;
+        for (int cc = 0; cc < 4; ++cc) {
+          const int c = col_half * 4 + cc;
           uint32_t v[32];
           if (args.mode == kEpiY) {
+            // lane j holds the scale of column col0 + j; shuffled to every row
+            const int64_t col0 = static_cast<int64_t>(nb) * BN + c * 32;
+            const float wl = (col0 + lane < args.N) ? __ldg(args.w_scale + col0 + lane) : 0.f;
             tmem_ld_32x32b_x32(dbuf + c * 32, v);
             tmem_ld_wait();
-            const float *ws = args.w_scale + col0;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float w = (col0 + j < args.N) ? __ldg(ws + j) : 0.f;
-              v[j] = __float_as_uint(
-                  __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j])), xs), w));
-            }
+            for (int j = 0; j < 32; ++j)
+              v[j] = __float_as_uint(__fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j])), xs),
+                                               __shfl_sync(0xffffffffu, wl, j)));
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0u;
@@ -346,20 +350,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_after();
       }
       // final pass: TMEM -> global
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c = col_half * 4 + cc;
         const int64_t col0 = static_cast<int64_t>(nb) * BN + c * 32;
         if (col0 >= args.N) break;
         const int nvalid = (col0 + 32 <= args.N) ? 32 : static_cast<int>(args.N - col0);
         uint32_t v[32];
         const bool zero = (args.mode == kEpiDelta) && !has_lora;
+        const float wl = (args.mode == kEpiY && !has_lora && col0 + lane < args.N)
+                             ? __ldg(args.w_scale + col0 + lane)
+                             : 0.f;
         if (!zero) {
           tmem_ld_32x32b_x32(dbuf + c * 32, v);
           tmem_ld_wait();
         }
-        if (!row_ok) continue;
         if (args.mode == kEpiY) {
           uint32_t packed[16];
-          const float *ws = args.w_scale + col0;
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
             float v0, v1;
@@ -367,20 +373,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               v0 = __uint_as_float(v[j]);
               v1 = __uint_as_float(v[j + 1]);
             } else {
-              const float w0 = (j < nvalid) ? __ldg(ws + j) : 0.f;
-              const float w1 = (j + 1 < nvalid) ? __ldg(ws + j + 1) : 0.f;
-              v0 = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j])), xs), w0);
-              v1 = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j + 1])), xs), w1);
+              v0 = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j])), xs),
+                             __shfl_sync(0xffffffffu, wl, j));
+              v1 = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j + 1])), xs),
+                             __shfl_sync(0xffffffffu, wl, j + 1));
             }
             __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
             packed[j / 2] = *reinterpret_cast<uint32_t *>(&h);
           }
+          if (!row_ok) continue;
           uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(args.out) + row * args.N + col0);
 #pragma unroll
           for (int t = 0; t < 4; ++t)
             if (t * 8 < nvalid)
               dst[t] = make_uint4(packed[4 * t], packed[4 * t + 1], packed[4 * t + 2], packed[4 * t + 3]);
         } else {
+          if (!row_ok) continue;
           uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint32_t *>(args.out) + row * args.N + col0);
 #pragma unroll
           for (int t = 0; t < 8; ++t)

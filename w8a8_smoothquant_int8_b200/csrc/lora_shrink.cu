@@ -26,12 +26,19 @@ namespace sq {
 constexpr int kShrinkWarps = 8;
 constexpr int kShrinkThreads = 32 * kShrinkWarps;
 
+// Two signed bytes of w (bytes `first_byte`, `first_byte`+1) -> packed bf16
+// pair, exactly.  The byte, biased by 128 (xor 0x80), is placed in the low
+// mantissa bits of 2^23 and 2^23 + 128 is subtracted; the result is a small
+// integer whose low 16 float bits are zero, so its bf16 pattern is the high
+// half of the float.  Needs only byte permutes and adds.
 __device__ __forceinline__ uint32_t bf16x2_of_s8(uint32_t w, int first_byte) {
-  // two consecutive signed bytes -> packed bf16 pair (exact)
-  const float lo = static_cast<float>(static_cast<int8_t>((w >> (8 * first_byte)) & 0xffu));
-  const float hi = static_cast<float>(static_cast<int8_t>((w >> (8 * first_byte + 8)) & 0xffu));
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t *>(&h);
+  const uint32_t wb = w ^ 0x80808080u;
+  const uint32_t magic = 0x4B000000u;
+  const uint32_t sel0 = 0x7650u | static_cast<uint32_t>(first_byte);
+  const uint32_t sel1 = 0x7650u | static_cast<uint32_t>(first_byte + 1);
+  const float f0 = __fsub_rn(__uint_as_float(__byte_perm(wb, magic, sel0)), 8388736.0f);
+  const float f1 = __fsub_rn(__uint_as_float(__byte_perm(wb, magic, sel1)), 8388736.0f);
+  return __byte_perm(__float_as_uint(f0), __float_as_uint(f1), 0x7632);
 }
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
@@ -60,7 +67,7 @@ __device__ __forceinline__ void shrink_warp_tile(const int8_t *__restrict__ Xq, 
   for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
     for (int t = 0; t < 4; ++t) acc[nt][t] = 0.f;
-  constexpr int kDepth = (kNT <= 4) ? 2 : 1;
+  constexpr int kDepth = (kNT <= 2) ? 4 : ((kNT <= 4) ? 2 : 1);
   for (int c0 = c_begin; c0 < nchunks; c0 += kDepth * c_step) {
     uint4 xa[kDepth], xb[kDepth], bv[kDepth][kNT][2];
 #pragma unroll
