@@ -66,6 +66,9 @@ typedef enum sq_dtype { SQ_DTYPE_F32 = 0, SQ_DTYPE_BF16 = 1 } sq_dtype;
 /* Largest packed LoRA width (sum over adapters of the rank rounded up to 16). */
 #define SQ_MAX_LORA_COLS 1024
 
+/* Largest rank of one adapter. */
+#define SQ_MAX_LORA_RANK 256
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *sq_status_string(int status);
 
@@ -129,7 +132,8 @@ int sq_quantize_weight(const uint16_t *W, const float *s, int64_t N, int64_t K,
  * path read the dequantized activations Xq*x_scale (which approximate X/s)
  * and still compute X*A^T; folding lora_alpha/r into B applies the LoRA
  * scaling once, offline.  This call writes adapter (A [r,K], B [N,r], both
- * bf16) at column offset `off` (a multiple of 16) of a pack of width R. */
+ * bf16, 1 <= r <= SQ_MAX_LORA_RANK) at column offset `off` (a multiple of 16)
+ * of a pack of width R. */
 int sq_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s, int64_t r,
                     int64_t K, int64_t N, float lora_alpha, int64_t R, int64_t off,
                     uint16_t *A_pack, uint16_t *B_pack, void *stream);
@@ -150,7 +154,8 @@ int sq_quant_act(const void *X, int x_dtype, const float *s, int64_t M, int64_t 
  * pack of width R (0 when R == 0). */
 size_t sq_linear_lora_workspace_size(int64_t M, int64_t R);
 
-/* Step 7 plus the LoRA delta, one launch sequence:
+/* Step 7 plus the LoRA delta, one launch sequence (M <= 64 tokens take a
+ * form built for streaming the weights; larger M the tensor-core tile form):
  *   Y[i,n] = bf16( f32(acc[i,n]) * x_scale_i * w_scale_n + delta[i,n] ),
  *   acc = Xq Wq^T (exact int32), delta[i,:] = (x_scale_i Xq[i,:] A_pack_a^T)
  *   B_pack_a^T for the adapter a of token i (none: delta = 0).

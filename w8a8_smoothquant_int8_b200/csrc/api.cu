@@ -48,8 +48,11 @@ struct Workspace {
   unsigned long long *mask;
 };
 
+// The large-M form needs the two T planes and the tile masks; the small-M
+// (decode) form needs its shrink partials.
 static size_t workspace_bytes(int64_t M, int64_t R) {
   if (R <= 0 || M <= 0) return 0;
+  if (decode_applicable(M)) return align256(decode_workspace_bytes(M));
   const size_t plane = align256(static_cast<size_t>(M) * static_cast<size_t>(R) * 2);
   return 2 * plane + align256(static_cast<size_t>((M + 127) / 128) * 8);
 }
@@ -180,7 +183,8 @@ int sq_quantize_weight(const uint16_t *W, const float *s, int64_t N, int64_t K, 
 int sq_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s, int64_t r, int64_t K,
                     int64_t N, float lora_alpha, int64_t R, int64_t off, uint16_t *A_pack,
                     uint16_t *B_pack, void *stream) {
-  if (r <= 0 || K < 0 || N < 0 || R <= 0 || off < 0) return SQ_ERR_INVALID_ARG;
+  if (r <= 0 || r > SQ_MAX_LORA_RANK || K < 0 || N < 0 || R <= 0 || off < 0)
+    return SQ_ERR_INVALID_ARG;
   if (K % 16 != 0 || K > SQ_MAX_K || R % 16 != 0 || R > SQ_MAX_LORA_COLS || off % 16 != 0)
     return SQ_ERR_UNSUPPORTED_SHAPE;
   const int64_t rpad = (r + 15) / 16 * 16;
@@ -235,6 +239,17 @@ static int linear_common(const int8_t *Xq, const float *x_scale, const int8_t *W
   if (K == 0 || (mode == 2 && !lora)) {
     // empty contraction (and no LoRA rows with K == 0 either: T = 0)
     return cuda_status(cudaMemsetAsync(out, 0, static_cast<size_t>(M) * N * esize, s));
+  }
+  if (decode_applicable(M)) {
+    // few tokens: bound by streaming the weights, see decode.cu
+    const bool timed = (mode == 0) && g_gemm_ev_before != nullptr;
+    if (timed && cudaEventRecord(g_gemm_ev_before, s) != cudaSuccess) return SQ_ERR_CUDA;
+    cudaError_t e = launch_decode(Xq, x_scale, Wq, w_scale, M, N, K, mode, A_pack, B_pack,
+                                  lora_offset, lora_rank, n_adapters, R, seg_offsets, seg_adapter,
+                                  S, lora ? static_cast<float *>(workspace) : nullptr, out, s);
+    if (e != cudaSuccess) return SQ_ERR_CUDA;
+    if (timed && cudaEventRecord(g_gemm_ev_after, s) != cudaSuccess) return SQ_ERR_CUDA;
+    return SQ_OK;
   }
   LoraOperands lo;
   LoraOperands *lop = nullptr;

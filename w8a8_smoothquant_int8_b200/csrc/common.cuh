@@ -48,6 +48,14 @@ cudaError_t launch_lora_shrink(const int8_t *Xq, const float *x_scale, int64_t M
                                const int32_t *seg_offsets, const int32_t *seg_adapter, int64_t S,
                                uint16_t *T_hi, uint16_t *T_lo, unsigned long long *mask,
                                cudaStream_t st);
+size_t decode_workspace_bytes(int64_t M);
+bool decode_applicable(int64_t M);
+cudaError_t launch_decode(const int8_t *Xq, const float *x_scale, const int8_t *Wq,
+                          const float *w_scale, int64_t M, int64_t N, int64_t K, int mode,
+                          const uint16_t *A_pack, const uint16_t *B_pack,
+                          const int32_t *lora_offset, const int32_t *lora_rank, int n_adapters,
+                          int64_t R, const int32_t *seg_offsets, const int32_t *seg_adapter,
+                          int64_t S, float *part, void *out, cudaStream_t st);
 cudaError_t launch_w8a8_gemm(const int8_t *Xq, const int8_t *Wq, const float *x_scale,
                              const float *w_scale, int64_t M, int64_t N, int64_t K, int mode,
                              void *out, const LoraOperands *lora, cudaStream_t st);

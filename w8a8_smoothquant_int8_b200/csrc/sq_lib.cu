@@ -3,4 +3,5 @@
 #include "quant.cu"
 #include "lora_shrink.cu"
 #include "gemm_sm100.cu"
+#include "decode.cu"
 #include "api.cu"
