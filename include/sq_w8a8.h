@@ -176,6 +176,30 @@ int sq_linear_lora(const int8_t *Xq, const float *x_scale, const int8_t *Wq,
                    int64_t S, uint16_t *Y, void *workspace, size_t workspace_bytes,
                    void *stream);
 
+/* Scratch size of sq_linear_lora_noalloc (bytes). */
+#define SQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* sq_linear_lora without a caller-provided workspace, for callers that cannot
+ * allocate device memory: code that runs inside an engine which plans every
+ * byte of device memory ahead and gives its plugins no allocator, or that
+ * must not call cudaMalloc at that point (it blocks the device and may fail
+ * under fragmentation).  The pages have no counterpart of this call.
+ * The scratch is one static device array of SQ_NOALLOC_SCRATCH_BYTES (16 MiB)
+ * that every GPU loading the library holds until the process exits; a call
+ * whose sq_linear_lora_workspace_size(M, R) exceeds it returns
+ * SQ_ERR_WORKSPACE.  The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress), so make that first call before any
+ * stream capture.  Each device has its own copy of the array and every call
+ * on that device uses it, keeping what the last call left there: calls that
+ * overlap on one GPU (for example on two streams) race, so serialize them.
+ * Other arguments, results and errors as sq_linear_lora.  Allocates nothing. */
+int sq_linear_lora_noalloc(const int8_t *Xq, const float *x_scale, const int8_t *Wq,
+                           const float *w_scale, int64_t M, int64_t N, int64_t K,
+                           const uint16_t *A_pack, const uint16_t *B_pack,
+                           const int32_t *lora_offset, const int32_t *lora_rank, int n_adapters,
+                           int64_t R, const int32_t *seg_offsets, const int32_t *seg_adapter,
+                           int64_t S, uint16_t *Y, void *stream);
+
 /* ---------------------------------------------------------------------------
  * Test entries: the same kernels with a different epilogue
  * ------------------------------------------------------------------------ */

@@ -21,7 +21,8 @@ __all__ = [
     "SQError", "LoraPack", "sq_status_string", "sq_version", "sq_device_supported",
     "sq_get_device_error", "sq_set_wait_timeout_ns", "sq_set_gemm_events", "sq_act_absmax_update", "sq_weight_absmax",
     "sq_compute_smoothing", "sq_quantize_weight", "sq_prepare_lora", "sq_quant_act",
-    "sq_linear_lora_workspace_size", "sq_linear_lora", "sq_gemm_i32", "sq_lora_delta",
+    "sq_linear_lora_workspace_size", "sq_linear_lora", "sq_linear_lora_noalloc", "sq_gemm_i32",
+    "sq_lora_delta",
 ]
 
 SQ_DTYPE_F32 = 0
@@ -199,6 +200,20 @@ def sq_linear_lora(Xq, x_scale, Wq, w_scale, lora: Optional[LoraPack], seg_offse
     _check(_lib().sq_linear_lora(_ptr(Xq), _ptr(x_scale), _ptr(Wq), _ptr(w_scale), M, N, K, a, b, o,
                                  r, n_ad, R, _ptr(seg_offsets), _ptr(seg_adapter), S, _ptr(Y), wp, wb,
                                  _stream(stream)), "sq_linear_lora")
+
+
+def sq_linear_lora_noalloc(Xq, x_scale, Wq, w_scale, lora: Optional[LoraPack], seg_offsets,
+                           seg_adapter, Y, stream=None) -> None:
+    """sq_linear_lora for callers that cannot allocate device memory: the
+    scratch is the library's static 16 MiB device array (shared by all calls,
+    so calls that overlap on the GPU race)."""
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    a, b, o, r, n_ad, R = _lora_args(lora)
+    S = 0 if seg_adapter is None else seg_adapter.shape[0]
+    _check(_lib().sq_linear_lora_noalloc(_ptr(Xq), _ptr(x_scale), _ptr(Wq), _ptr(w_scale), M, N, K,
+                                         a, b, o, r, n_ad, R, _ptr(seg_offsets), _ptr(seg_adapter),
+                                         S, _ptr(Y), _stream(stream)), "sq_linear_lora_noalloc")
 
 
 def sq_gemm_i32(Xq, Wq, acc, stream=None) -> None:

@@ -35,6 +35,8 @@ SIGNATURES = {
     "sq_linear_lora_workspace_size": ([I64, I64], SZ),
     "sq_linear_lora": ([P, P, P, P, I64, I64, I64, P, P, P, P, I32, I64, P, P, I64, P, P, SZ, P],
                        I32),
+    "sq_linear_lora_noalloc": ([P, P, P, P, I64, I64, I64, P, P, P, P, I32, I64, P, P, I64, P, P],
+                               I32),
     "sq_gemm_i32": ([P, P, I64, I64, I64, P, P], I32),
     "sq_lora_delta": ([P, P, I64, I64, I64, P, P, P, P, I32, I64, P, P, I64, P, P, SZ, P], I32),
 }

@@ -87,6 +87,9 @@ static int check_lora_args(int64_t M, int64_t K, const uint16_t *A_pack, const u
 
 using namespace sq;
 
+// capability of the current device (cached), for the entry points below
+static int sq_device_supported_current() { return check_device(); }
+
 extern "C" {
 
 const char *sq_status_string(int status) {

@@ -5,3 +5,4 @@
 #include "gemm_sm100.cu"
 #include "decode.cu"
 #include "api.cu"
+#include "noalloc.cu"
