@@ -56,6 +56,29 @@ def parse():
     return p.parse_args()
 
 
+# DRAM bytes (read + write) of one fused-GEMM launch on the default workload,
+# from the ncu capture summarised in profiles/w8a8_lora_gemm_llama3_8b_qkv_m2048.md.
+# It describes that kernel source only: any other source reports null.
+GEMM_TRAFFIC = {
+    "source_sha256": "bee6e824e4d901f6fce1015910c7733fa3c901d81d406bce5204199274df0d78",
+    "workload": DEFAULT_WORKLOAD,
+    "bytes": 33993984 + 430080,
+}
+
+
+def gemm_traffic(workload: str):
+    import hashlib
+    src = os.path.join(ROOT, "w8a8_smoothquant_int8_b200", "csrc", "gemm_sm100.cu")
+    try:
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    if sha != GEMM_TRAFFIC["source_sha256"] or workload != GEMM_TRAFFIC["workload"]:
+        return None
+    return GEMM_TRAFFIC["bytes"]
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -365,7 +388,8 @@ def run_ours(args):
         "roofline": {"bound": "tensor", "kernel": "w8a8_lora_gemm_kernel", "achieved": gemm_tops,
                      "peak": int8_peak, "unit": "TOPS", "frac": gemm_tops / int8_peak,
                      "peak_source": f"{peak_kind}: 2 x bf16 burst {peaks['bf16_tflops']} TFLOP/s",
-                     "gemm_us": gemm_avg_s * 1e6, "traffic": None,
+                     "gemm_us": gemm_avg_s * 1e6, "traffic": gemm_traffic(wl.spec.name),
+                     "traffic_unit": "bytes per launch (ncu dram read+write)",
                      "algorithmic_ops": ops_step},
         "cpu_baseline": cpu,
         "e2e": e2e,
