@@ -95,6 +95,24 @@ def lora_flops(wl) -> int:
 
 
 # ---------------------------------------------------------------------------
+# ranks: every rank runs a replica; times are maxed over ranks
+# ---------------------------------------------------------------------------
+def reduce_max(values, device=None):
+    """Element-wise maximum of `values` over all ranks (identity with one process)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def job_tops(ops_per_step: int, steps: int, world: int, total_ms: float) -> float:
+    """Whole-job throughput: the work of every rank over the slowest rank's time."""
+    return ops_per_step * steps * world / (total_ms * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
@@ -320,10 +338,7 @@ def run_ours(args):
     clocks = sampler.stop()
     step_ms = [e[0].elapsed_time(e[1]) for e in ev]
     gemm_ms = [e[2].elapsed_time(e[3]) for e in ev]
-    t_local = torch.tensor([sum(step_ms), sum(gemm_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
-    t_step_total, t_gemm_total = [float(x) for x in t_local.cpu()]
+    t_step_total, t_gemm_total = reduce_max([sum(step_ms), sum(gemm_ms)], dev)
     err = sq.sq_get_device_error(clear=True)
     if err:
         raise SystemExit(f"device error {err}: {sq.sq_status_string(err)}")
@@ -346,19 +361,16 @@ def run_ours(args):
         torch.cuda.synchronize()
         if i >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
-    t_e2e = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
-    t_e2e = float(t_e2e.item())
+    t_e2e = reduce_max([sum(e2e_ms)], dev)[0]
     e2e = None
     if e2e_ms:
-        e2e = {"value": 2 * M * N * K * len(e2e_ms) * world / (t_e2e * 1e-3) / 1e12, "unit": "TOPS",
+        e2e = {"value": job_tops(2 * M * N * K, len(e2e_ms), world, t_e2e), "unit": "TOPS",
                "h2d_bytes_per_step": int(X_host.numel() * X_host.element_size()),
                "d2h_bytes_per_step": int(Y_host.numel() * Y_host.element_size()),
                "ms_per_step": t_e2e / len(e2e_ms)}
 
     ops_step = 2 * M * N * K
-    value = ops_step * n * world / (t_step_total * 1e-3) / 1e12
+    value = job_tops(ops_step, n, world, t_step_total)
     tok_s = M * n * world / (t_step_total * 1e-3)
     gemm_avg_s = t_gemm_total * 1e-3 / n
     gemm_tops = ops_step / gemm_avg_s / 1e12

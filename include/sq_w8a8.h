@@ -86,8 +86,17 @@ int sq_get_device_error(int *code, int clear);
 
 /* Upper bound, in nanoseconds, of every spin-wait inside the kernels
  * (default 2 s).  A wait that runs out makes the kernel stop, record
- * SQ_ERR_DEVICE_TIMEOUT and return.  Host-side setting for later launches. */
+ * SQ_ERR_DEVICE_TIMEOUT and return.  Bounds below 1 us (finer than the
+ * device timer) make a wait give up after one non-blocking probe.  Host-side
+ * setting for later launches. */
 int sq_set_wait_timeout_ns(uint64_t ns);
+
+/* Test of failure detection: launches one block that waits, with the bound
+ * `timeout_ns` (1 ns .. 100 ms), on a barrier nothing ever arrives on.  The
+ * wait gives up and SQ_ERR_DEVICE_TIMEOUT is recorded for
+ * sq_get_device_error(); the context stays usable.  Returns the launch
+ * status. */
+int sq_selftest_wait_timeout(uint64_t timeout_ns, void *stream);
 
 /* Measurement aid: when both are non-NULL, sq_linear_lora records the
  * cudaEvent_t `before` on its stream right before it launches the fused GEMM

@@ -19,7 +19,7 @@ from . import _native
 
 __all__ = [
     "SQError", "LoraPack", "sq_status_string", "sq_version", "sq_device_supported",
-    "sq_get_device_error", "sq_set_wait_timeout_ns", "sq_set_gemm_events", "sq_act_absmax_update", "sq_weight_absmax",
+    "sq_get_device_error", "sq_set_wait_timeout_ns", "sq_set_gemm_events", "sq_selftest_wait_timeout", "sq_act_absmax_update", "sq_weight_absmax",
     "sq_compute_smoothing", "sq_quantize_weight", "sq_prepare_lora", "sq_quant_act",
     "sq_linear_lora_workspace_size", "sq_linear_lora", "sq_linear_lora_noalloc", "sq_gemm_i32",
     "sq_lora_delta",
@@ -91,6 +91,11 @@ def sq_get_device_error(clear: bool = True) -> int:
 
 def sq_set_wait_timeout_ns(ns: int) -> None:
     _check(_lib().sq_set_wait_timeout_ns(int(ns)), "sq_set_wait_timeout_ns")
+
+
+def sq_selftest_wait_timeout(timeout_ns: int, stream=None) -> None:
+    """Launch a bounded wait on a barrier nothing arrives on (failure-detection test)."""
+    _check(_lib().sq_selftest_wait_timeout(int(timeout_ns), _stream(stream)), "sq_selftest_wait_timeout")
 
 
 def sq_set_gemm_events(before=None, after=None) -> None:

@@ -26,6 +26,7 @@ SIGNATURES = {
     "sq_get_device_error": ([ctypes.POINTER(I32), I32], I32),
     "sq_set_wait_timeout_ns": ([U64], I32),
     "sq_set_gemm_events": ([P, P], I32),
+    "sq_selftest_wait_timeout": ([U64, P], I32),
     "sq_act_absmax_update": ([P, I32, I64, I64, P, P], I32),
     "sq_weight_absmax": ([P, I64, I64, P, P], I32),
     "sq_compute_smoothing": ([P, P, I64, F32, P, P], I32),

@@ -4,6 +4,7 @@
 #include <cstring>
 
 #include "common.cuh"
+#include "ptx_sm100.cuh"
 
 namespace sq {
 
@@ -85,6 +86,23 @@ static int check_lora_args(int64_t M, int64_t K, const uint16_t *A_pack, const u
 
 }  // namespace sq
 
+namespace sq {
+// A wait on an mbarrier that nothing ever arrives on: the bounded wait used
+// by every kernel must give up and record SQ_ERR_DEVICE_TIMEOUT.
+__global__ void selftest_wait_kernel(uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, timeout_ns, &abort_flag))
+    record_device_error(SQ_ERR_DEVICE_TIMEOUT);
+}
+}  // namespace sq
+
 using namespace sq;
 
 // capability of the current device (cached), for the entry points below
@@ -140,6 +158,14 @@ int sq_set_gemm_events(void *before, void *after) {
   g_gemm_ev_before = static_cast<cudaEvent_t>(before);
   g_gemm_ev_after = static_cast<cudaEvent_t>(after);
   return SQ_OK;
+}
+
+int sq_selftest_wait_timeout(uint64_t timeout_ns, void *stream) {
+  if (timeout_ns == 0 || timeout_ns > 100000000ull) return SQ_ERR_INVALID_ARG;
+  int st = check_device();
+  if (st) return st;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+  return cuda_status(cudaGetLastError());
 }
 
 int sq_act_absmax_update(const void *X, int x_dtype, int64_t M, int64_t K, float *act_absmax,

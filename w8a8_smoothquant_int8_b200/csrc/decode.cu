@@ -212,7 +212,9 @@ __global__ void __launch_bounds__(kDecGemmThreads) decode_gemm_kernel(
     int st = 0;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
-      if (!(ok = mbar_wait(&ctl.full[st], phase, timeout_ns, abort_flag))) break;
+      // the warp leaves together: the mma.sync below needs all lanes
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ctl.full[st], phase, timeout_ns, abort_flag))))
+        break;
       const uint8_t *wt = ring + st * kDecStageBytes;
       const uint8_t *xt = wt + kDecWBytes;
 #pragma unroll

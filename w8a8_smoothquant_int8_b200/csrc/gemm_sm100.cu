@@ -315,7 +315,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int mb, nb;
       tile_coords(tile, args, mb, nb);
       const bool has_lora = use_lora && tile_lora_mask(args, mb) != 0ull;
-      if (!(ok = mbar_wait(&ctl->acc_full[b], (i >> 1) & 1, args.timeout_ns, abort_flag))) break;
+      // the warp leaves together: the collective TMEM loads below need all lanes
+      if (!(ok = __all_sync(0xffffffffu,
+                            mbar_wait(&ctl->acc_full[b], (i >> 1) & 1, args.timeout_ns, abort_flag))))
+        break;
       tc_fence_after();
       const int64_t row = static_cast<int64_t>(mb) * BM + row_in_tile;
       const bool row_ok = row < args.M;
@@ -344,7 +347,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive_cluster(base_ready_pair + 8u * b);
-        if (!(ok = mbar_wait(&ctl->lora_done[b], lora_uses[b] & 1u, args.timeout_ns, abort_flag)))
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ctl->lora_done[b], lora_uses[b] & 1u,
+                                                      args.timeout_ns, abort_flag))))
           break;
         ++lora_uses[b];
         tc_fence_after();
