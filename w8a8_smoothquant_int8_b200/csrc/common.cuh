@@ -19,6 +19,20 @@ __device__ __forceinline__ void record_device_error(unsigned int code) {
 // Default bound of every device-side spin-wait (ns), settable from the host.
 uint64_t wait_timeout_ns();
 
+// Number of SMs of the current device (cached per device).
+static inline int sm_count_of_current_device() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
 // LoRA operands of the fused GEMM: T planes [M,R] bf16 (written by the
 // shrink kernel), the packed B [N,R] bf16 and one 16-column-group mask per
 // 128-token tile.

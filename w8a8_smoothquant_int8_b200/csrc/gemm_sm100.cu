@@ -457,18 +457,6 @@ static bool make_tmap(CUtensorMap *m, const void *base, CUtensorMapDataType dt, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static int sm_count_of_current_device() {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int n = 0;
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = n > 0 ? n : 148;
-  }
-  return cached[dev];
-}
 
 // Launch the fused GEMM.  `lora` may be null (plain W8A8 / raw int32).
 cudaError_t launch_w8a8_gemm(const int8_t *Xq, const int8_t *Wq, const float *x_scale,
