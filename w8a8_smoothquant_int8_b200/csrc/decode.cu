@@ -19,6 +19,7 @@
 
 #include "common.cuh"
 #include "ptx_sm100.cuh"
+#include "tmap.cuh"
 
 namespace sq {
 
@@ -117,7 +118,7 @@ constexpr int kDecGemmThreads = 32 * (kDecComputeWarps + 1);
 
 __device__ __forceinline__ void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                              uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 "
       "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
@@ -226,13 +227,17 @@ __global__ void __launch_bounds__(kDecGemmThreads) decode_gemm_kernel(
         const uint4 xb = *reinterpret_cast<const uint4 *>(xt + rb * 128 + (((4 * h + tig) ^ (rb & 7)) * 16));
         const uint32_t fa0[4] = {xa.x, xb.x, xa.y, xb.y};
         const uint32_t fa1[4] = {xa.z, xb.z, xa.w, xb.w};
+        uint4 bw[2];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
           const int row = nh * 16 + nt * 8 + g;
-          const uint4 bw = *reinterpret_cast<const uint4 *>(wt + row * 128 + (((4 * h + tig) ^ (row & 7)) * 16));
-          mma_s8_16832(acc[nt], fa0, bw.x, bw.y);
-          mma_s8_16832(acc[nt], fa1, bw.z, bw.w);
+          bw[nt] = *reinterpret_cast<const uint4 *>(wt + row * 128 + (((4 * h + tig) ^ (row & 7)) * 16));
         }
+        // independent accumulators back to back
+        mma_s8_16832(acc[0], fa0, bw[0].x, bw[0].y);
+        mma_s8_16832(acc[1], fa0, bw[1].x, bw[1].y);
+        mma_s8_16832(acc[0], fa1, bw[0].z, bw[0].w);
+        mma_s8_16832(acc[1], fa1, bw[1].z, bw[1].w);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.empty[st]);
