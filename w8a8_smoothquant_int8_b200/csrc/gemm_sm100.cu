@@ -50,6 +50,10 @@ constexpr int kThreads = 320;        // producer warp, MMA warp, 8 epilogue warp
 constexpr int kEpiWarps = 8;         // two per TMEM lane quarter, each owning 128 columns
 constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;  // two 256-column accumulator buffers
+// Output staging of the bf16 epilogue: per epilogue warp two buffers of 32
+// rows x 32 columns (64-byte swizzle), written to global by TMA stores.
+constexpr int kEpiBufBytes = 32 * 32 * 2;
+constexpr int kEpiSmem = kEpiWarps * 2 * kEpiBufBytes;  // 32 KB
 // Bound of the final waits for this CTA's own copies and MMAs, independent of
 // the (possibly tiny) user wait bound: those always complete.
 constexpr uint64_t kDrainNs = 1000000000ull;
@@ -79,7 +83,9 @@ struct SharedCtl {
   int abort;
 };
 
-constexpr size_t kSmemBytes = static_cast<size_t>(kStages) * kStageBytes + sizeof(SharedCtl) + 1024;
+static_assert(sizeof(SharedCtl) <= 1024, "control block fits its 1 KB slot");
+// stages | control block (1 KB slot) | output staging | alignment slack
+constexpr size_t kSmemBytes = static_cast<size_t>(kStages) * kStageBytes + 1024 + kEpiSmem + 1024;
 
 __device__ __forceinline__ void tile_coords(int tile, const GemmArgs &a, int &mb, int &nb) {
   // groups of group_m token tiles walk the output-channel tiles together, so
@@ -100,6 +106,35 @@ __device__ __forceinline__ unsigned long long tile_lora_mask(const GemmArgs &a, 
   unsigned long long m = a.lora_mask[h0];
   if (h1 < nh) m |= a.lora_mask[h1];
   return m;
+}
+
+// Scales of the columns col0 .. col0+31, the same in every lane (warp-uniform
+// 16-byte loads; the columns past N read as 0).
+__device__ __forceinline__ void load_wscale32(const float *__restrict__ w, int64_t col0, int64_t N,
+                                              float (&ws)[32]) {
+  if (col0 + 32 <= N) {
+    const float4 *p = reinterpret_cast<const float4 *>(w + col0);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 t = __ldg(p + q);
+      ws[4 * q] = t.x; ws[4 * q + 1] = t.y; ws[4 * q + 2] = t.z; ws[4 * q + 3] = t.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) ws[j] = (col0 + j < N) ? __ldg(w + col0 + j) : 0.f;
+  }
+}
+
+// Dequantized values of 32 accumulators: RN(RN(float(acc) * xs) * w_j).
+__device__ __forceinline__ void dequant32(uint32_t (&v)[32], float xs, const float (&ws)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    const float2 f = make_float2(__int2float_rn(static_cast<int>(v[j])),
+                                 __int2float_rn(static_cast<int>(v[j + 1])));
+    const float2 y = __fmul2_rn(__fmul2_rn(f, make_float2(xs, xs)), make_float2(ws[j], ws[j + 1]));
+    v[j] = __float_as_uint(y.x);
+    v[j + 1] = __float_as_uint(y.y);
+  }
 }
 
 __device__ __forceinline__ void signal_abort(SharedCtl *ctl) {
@@ -156,11 +191,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                           const __grid_constant__ CUtensorMap tm_wq,
                           const __grid_constant__ CUtensorMap tm_thi,
                           const __grid_constant__ CUtensorMap tm_tlo,
-                          const __grid_constant__ CUtensorMap tm_bp, const GemmArgs args) {
+                          const __grid_constant__ CUtensorMap tm_bp,
+                          const __grid_constant__ CUtensorMap tm_y, const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   SharedCtl *ctl = reinterpret_cast<SharedCtl *>(smem + kStages * kStageBytes);
+  uint8_t *epi_smem = smem + kStages * kStageBytes + 1024;
   volatile int *abort_flag = &ctl->abort;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -310,6 +347,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t lora_uses[2] = {0, 0};
     bool ok = true;
     int i = 0;
+    int sbuf = 0;  // output staging buffer of this warp
     for (int tile = pair; tile < args.num_tiles; tile += args.num_pairs, ++i) {
       const int b = i & 1;
       const uint32_t dbuf = tmem + static_cast<uint32_t>(b) * 256u + lane_addr;
@@ -330,15 +368,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int c = col_half * 4 + cc;
           uint32_t v[32];
           if (args.mode == kEpiY) {
-            // lane j holds the scale of column col0 + j; shuffled to every row
             const int64_t col0 = static_cast<int64_t>(nb) * BN + c * 32;
-            const float wl = (col0 + lane < args.N) ? __ldg(args.w_scale + col0 + lane) : 0.f;
+            float ws[32];
+            load_wscale32(args.w_scale, col0, args.N, ws);
             tmem_ld_32x32b_x32(dbuf + c * 32, v);
             tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              v[j] = __float_as_uint(__fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j])), xs),
-                                               __shfl_sync(0xffffffffu, wl, j)));
+            dequant32(v, xs, ws);
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0u;
@@ -362,36 +397,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int nvalid = (col0 + 32 <= args.N) ? 32 : static_cast<int>(args.N - col0);
         uint32_t v[32];
         const bool zero = (args.mode == kEpiDelta) && !has_lora;
-        const float wl = (args.mode == kEpiY && !has_lora && col0 + lane < args.N)
-                             ? __ldg(args.w_scale + col0 + lane)
-                             : 0.f;
         if (!zero) {
           tmem_ld_32x32b_x32(dbuf + c * 32, v);
           tmem_ld_wait();
         }
         if (args.mode == kEpiY) {
+          if (!has_lora) {
+            float ws[32];
+            load_wscale32(args.w_scale, col0, args.N, ws);
+            dequant32(v, xs, ws);
+          }
           uint32_t packed[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            float v0, v1;
-            if (has_lora) {
-              v0 = __uint_as_float(v[j]);
-              v1 = __uint_as_float(v[j + 1]);
-            } else {
-              v0 = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j])), xs),
-                             __shfl_sync(0xffffffffu, wl, j));
-              v1 = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(v[j + 1])), xs),
-                             __shfl_sync(0xffffffffu, wl, j + 1));
-            }
-            __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+            __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
             packed[j / 2] = *reinterpret_cast<uint32_t *>(&h);
           }
-          if (!row_ok) continue;
-          uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(args.out) + row * args.N + col0);
+          // stage the warp's 32 rows x 32 columns, then one TMA store (rows
+          // past M and columns past N are clipped by the store)
+          uint8_t *sb = epi_smem + (ew * 2 + sbuf) * kEpiBufBytes;
+          if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read it
+          __syncwarp();
 #pragma unroll
           for (int t = 0; t < 4; ++t)
-            if (t * 8 < nvalid)
-              dst[t] = make_uint4(packed[4 * t], packed[4 * t + 1], packed[4 * t + 2], packed[4 * t + 3]);
+            *reinterpret_cast<uint4 *>(sb + lane * 64 + ((t ^ ((lane >> 1) & 3)) * 16)) =
+                make_uint4(packed[4 * t], packed[4 * t + 1], packed[4 * t + 2], packed[4 * t + 3]);
+          fence_proxy_async_shared();
+          __syncwarp();
+          const int64_t row_base = static_cast<int64_t>(mb) * BM + rank * kHalf + quarter * 32;
+          if (lane == 0 && row_base < args.M) {
+            tma_store_2d(&tm_y, sb, static_cast<int32_t>(col0), static_cast<int32_t>(row_base));
+            bulk_commit_group();
+          }
+          sbuf ^= 1;
         } else {
           if (!row_ok) continue;
           uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint32_t *>(args.out) + row * args.N + col0);
@@ -406,6 +444,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_arrive_cluster(acc_empty_pair + 8u * b);
     }
     if (!ok) signal_abort(ctl);
+    if (lane == 0) bulk_wait_group<0>();  // this warp's output stores are complete
   }
 
   if (*abort_flag) {
@@ -431,7 +470,11 @@ cudaError_t launch_w8a8_gemm(const int8_t *Xq, const int8_t *Wq, const float *x_
                              const float *w_scale, int64_t M, int64_t N, int64_t K, int mode,
                              void *out, const LoraOperands *lora, cudaStream_t st) {
   if (M == 0 || N == 0) return cudaSuccess;
-  CUtensorMap tm_xq, tm_wq, tm_thi, tm_tlo, tm_bp;
+  CUtensorMap tm_xq, tm_wq, tm_thi, tm_tlo, tm_bp, tm_y;
+  memset(&tm_y, 0, sizeof tm_y);
+  if (mode == kEpiY && !make_tmap(&tm_y, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, 32, 32,
+                                  CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
   memset(&tm_thi, 0, sizeof tm_thi);
   memset(&tm_tlo, 0, sizeof tm_tlo);
   memset(&tm_bp, 0, sizeof tm_bp);
@@ -475,7 +518,7 @@ cudaError_t launch_w8a8_gemm(const int8_t *Xq, const int8_t *Wq, const float *x_
     attr_set = true;
   }
   w8a8_lora_gemm_kernel<<<2 * a.num_pairs, kThreads, kSmemBytes, st>>>(tm_xq, tm_wq, tm_thi, tm_tlo,
-                                                                       tm_bp, a);
+                                                                       tm_bp, tm_y, a);
   return cudaGetLastError();
 }
 
