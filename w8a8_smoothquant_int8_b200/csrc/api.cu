@@ -49,13 +49,13 @@ struct Workspace {
   unsigned long long *mask;
 };
 
-// The large-M form needs the two T planes and the tile masks; the small-M
+// The large-M form needs the two T planes and one mask word per 16 tokens; the small-M
 // (decode) form needs its shrink partials.
 static size_t workspace_bytes(int64_t M, int64_t R) {
   if (R <= 0 || M <= 0) return 0;
   if (decode_applicable(M)) return align256(decode_workspace_bytes(M));
   const size_t plane = align256(static_cast<size_t>(M) * static_cast<size_t>(R) * 2);
-  return 2 * plane + align256(static_cast<size_t>((M + 127) / 128) * 8);
+  return 2 * plane + align256(static_cast<size_t>((M + 15) / 16) * 8);
 }
 
 static Workspace carve(void *ws, int64_t M, int64_t R) {

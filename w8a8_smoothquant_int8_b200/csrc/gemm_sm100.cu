@@ -66,7 +66,7 @@ struct GemmArgs {
   const float *x_scale;
   const float *w_scale;
   void *out;
-  const unsigned long long *lora_mask;  // [ceil(M/128)] 16-column group masks, or null
+  const unsigned long long *lora_mask;  // [ceil(M/16)] 16-column group masks, or null
   int num_mb, num_nb, num_tiles, group_m, num_pairs;
   uint64_t timeout_ns;
 };
@@ -99,12 +99,16 @@ __device__ __forceinline__ void tile_coords(int tile, const GemmArgs &a, int &mb
   nb = local / gm;
 }
 
+// The 16-column groups of R that the tile's tokens use: the OR of the words
+// of its groups of 16 tokens.
 __device__ __forceinline__ unsigned long long tile_lora_mask(const GemmArgs &a, int mb) {
   if (a.lora_mask == nullptr || a.mode == kEpiAcc) return 0ull;
-  const int h0 = 2 * mb, h1 = 2 * mb + 1;  // the two 128-token halves
-  const int nh = static_cast<int>((a.M + 127) / 128);
-  unsigned long long m = a.lora_mask[h0];
-  if (h1 < nh) m |= a.lora_mask[h1];
+  const int g0 = mb * (BM / 16);
+  const int ng = static_cast<int>((a.M + 15) / 16);
+  unsigned long long m = 0ull;
+#pragma unroll
+  for (int g = 0; g < BM / 16; ++g)
+    if (g0 + g < ng) m |= __ldg(a.lora_mask + g0 + g);
   return m;
 }
 
@@ -239,6 +243,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __syncthreads();
   cluster_sync();  // both CTAs' barriers exist before any remote arrive or copy
   tc_fence_after();
+  // inputs written by the preceding kernels are read only from here on
+  // (programmatic dependent launch: the set-up above may overlap their tail)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const uint32_t tmem = ctl->tmem_base;
 
   if (warp == 0) {
@@ -517,9 +524,17 @@ cudaError_t launch_w8a8_gemm(const int8_t *Xq, const int8_t *Wq, const float *x_
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  w8a8_lora_gemm_kernel<<<2 * a.num_pairs, kThreads, kSmemBytes, st>>>(tm_xq, tm_wq, tm_thi, tm_tlo,
-                                                                       tm_bp, tm_y, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * a.num_pairs, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, w8a8_lora_gemm_kernel, tm_xq, tm_wq, tm_thi, tm_tlo, tm_bp, tm_y, a);
 }
 
 }  // namespace sq

@@ -8,8 +8,8 @@
 // T_lo = bf16(T - T_hi), with zeros outside the token's adapter columns, so
 // that the GEMM epilogue can apply every adapter of a 128-token tile with
 // dense bf16 tensor-core MMAs and still carry ~16 significant bits of T.
-// mask[tile] collects, per 128-token tile, the 16-column groups of R that
-// some token of the tile uses.
+// mask[g] holds, per group of 16 tokens, the 16-column groups of R that some
+// token of the group uses (each word written once, by the block of the group).
 //
 // The contraction is a skinny GEMM (N = rank <= 64 per pass) done with
 // warp-level bf16 tensor-core MMAs (m16n8k16, fp32 accumulation): the int8
@@ -174,8 +174,11 @@ __global__ void __launch_bounds__(kShrinkThreads) lora_shrink_kernel(
   }
   __syncthreads();
   if (row0 >= M) return;  // whole row group; only group barriers follow
+  // the codes and scales come from the preceding kernel (a no-op unless this
+  // grid is launched as a programmatic dependent)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // zero both planes for the group's rows, and set the tile mask
+  // zero both planes for the group's rows, and write the group's mask word
   {
     const int64_t nrows = (M - row0 < 16) ? (M - row0) : 16;
     const int64_t words = nrows * R / 8;  // 16-byte words (R % 16 == 0)
@@ -191,7 +194,7 @@ __global__ void __launch_bounds__(kShrinkThreads) lora_shrink_kernel(
         const int off = s_off[rg][r], rpad = (s_rank[rg][r] + 15) & ~15;
         for (int gi = off / 16; gi < (off + rpad) / 16; ++gi) bits |= 1ull << gi;
       }
-      if (bits) atomicOr(mask + (row0 >> 7), bits);
+      mask[row0 >> 4] = bits;
     }
   }
   group_sync(rg, kKS);
@@ -263,6 +266,9 @@ __global__ void __launch_bounds__(kShrinkThreads) lora_shrink_kernel(
     }
     done |= rows_a;
   }
+  // the following kernel may start its set-up once every block is here (not
+  // earlier, so that it does not hold SMs that later blocks of this one need)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 cudaError_t launch_lora_shrink(const int8_t *Xq, const float *x_scale, int64_t M, int64_t K,
@@ -272,28 +278,40 @@ cudaError_t launch_lora_shrink(const int8_t *Xq, const float *x_scale, int64_t M
                                uint16_t *T_hi, uint16_t *T_lo, unsigned long long *mask,
                                cudaStream_t st) {
   if (M == 0) return cudaSuccess;
-  cudaError_t e = cudaMemsetAsync(mask, 0, static_cast<size_t>((M + 127) / 128) * 8, st);
-  if (e != cudaSuccess) return e;
   const int64_t row_tiles = (M + 15) / 16;
-  // widest row grouping that still leaves about two blocks per SM
+  // widest row grouping that still leaves about two blocks per SM.  Launched
+  // in plain stream order: as a programmatic dependent of the quantizer its
+  // blocks were placed worse on the large workloads (measured); the fused
+  // GEMM that follows is launched as its dependent instead.
   const unsigned g1 = static_cast<unsigned>(row_tiles);
-  if (row_tiles >= 8 * 2 * 148)
-    lora_shrink_kernel<8><<<(g1 + 7) / 8, kShrinkThreads, 0, st>>>(
-        Xq, x_scale, M, K, A_pack, lora_offset, lora_rank, n_adapters, R, seg_offsets, seg_adapter,
-        S, T_hi, T_lo, mask);
-  else if (row_tiles >= 4 * 2 * 148)
-    lora_shrink_kernel<4><<<(g1 + 3) / 4, kShrinkThreads, 0, st>>>(
-        Xq, x_scale, M, K, A_pack, lora_offset, lora_rank, n_adapters, R, seg_offsets, seg_adapter,
-        S, T_hi, T_lo, mask);
-  else if (row_tiles >= 2 * 2 * 148)
-    lora_shrink_kernel<2><<<(g1 + 1) / 2, kShrinkThreads, 0, st>>>(
-        Xq, x_scale, M, K, A_pack, lora_offset, lora_rank, n_adapters, R, seg_offsets, seg_adapter,
-        S, T_hi, T_lo, mask);
-  else
-    lora_shrink_kernel<1><<<g1, kShrinkThreads, 0, st>>>(
-        Xq, x_scale, M, K, A_pack, lora_offset, lora_rank, n_adapters, R, seg_offsets, seg_adapter,
-        S, T_hi, T_lo, mask);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kShrinkThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  if (row_tiles >= 8 * 2 * 148) {
+    cfg.gridDim = dim3((g1 + 7) / 8, 1, 1);
+    return cudaLaunchKernelEx(&cfg, lora_shrink_kernel<8>, Xq, x_scale, M, K, A_pack, lora_offset,
+                              lora_rank, n_adapters, R, seg_offsets, seg_adapter, S, T_hi, T_lo,
+                              mask);
+  }
+  if (row_tiles >= 4 * 2 * 148) {
+    cfg.gridDim = dim3((g1 + 3) / 4, 1, 1);
+    return cudaLaunchKernelEx(&cfg, lora_shrink_kernel<4>, Xq, x_scale, M, K, A_pack, lora_offset,
+                              lora_rank, n_adapters, R, seg_offsets, seg_adapter, S, T_hi, T_lo,
+                              mask);
+  }
+  if (row_tiles >= 2 * 2 * 148) {
+    cfg.gridDim = dim3((g1 + 1) / 2, 1, 1);
+    return cudaLaunchKernelEx(&cfg, lora_shrink_kernel<2>, Xq, x_scale, M, K, A_pack, lora_offset,
+                              lora_rank, n_adapters, R, seg_offsets, seg_adapter, S, T_hi, T_lo,
+                              mask);
+  }
+  cfg.gridDim = dim3(g1, 1, 1);
+  return cudaLaunchKernelEx(&cfg, lora_shrink_kernel<1>, Xq, x_scale, M, K, A_pack, lora_offset,
+                            lora_rank, n_adapters, R, seg_offsets, seg_adapter, S, T_hi, T_lo,
+                            mask);
 }
 
 }  // namespace sq
