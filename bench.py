@@ -60,9 +60,9 @@ def parse():
 # from the ncu capture summarised in profiles/w8a8_lora_gemm_llama3_8b_qkv_m2048.md.
 # It describes that kernel source only: any other source reports null.
 GEMM_TRAFFIC = {
-    "source_sha256": "bee6e824e4d901f6fce1015910c7733fa3c901d81d406bce5204199274df0d78",
+    "source_sha256": "c6429fb71707a01faa20e1b0b08fb3c3b2e7410a0fc50376fb111933d2470d6c",
     "workload": DEFAULT_WORKLOAD,
-    "bytes": 33993984 + 430080,
+    "bytes": 34068992 + 1645824,
 }
 
 
