@@ -7,7 +7,8 @@
 //   kernel 1 (shrink)   one warp per (token, K slice): partial sums of
 //                       T[i,:] = x_scale_i * Xq[i,:] A_a^T over the slice,
 //                       written to a scratch table (no atomics: the sums are
-//                       later added in a fixed order);
+//                       later added in a fixed order); it lets the GEMM grid
+//                       launch at once, so the weight stream overlaps it;
 //   kernel 2 (GEMM + expand), one block per 32 output channels:
 //                       acc = Xq Wq^T with int8 tensor-core MMAs (m16n8k32,
 //                       exact int32) from a TMA-fed ring of Wq tiles; then,
@@ -32,12 +33,16 @@ constexpr int kDecThreads = 256;
 // ---------------------------------------------------------------------------
 // kernel 1: shrink partials.  part[(i * kDecKSplit + ks) * kDecMaxRank + j]
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kDecThreads) decode_shrink_kernel(
+__global__ void __launch_bounds__(kDecThreads, 1) decode_shrink_kernel(
     const int8_t *__restrict__ Xq, const float *__restrict__ x_scale, int64_t M, int64_t K,
     const uint16_t *__restrict__ A_pack, const int32_t *__restrict__ lora_offset,
     const int32_t *__restrict__ lora_rank, int n_adapters, int64_t R,
     const int32_t *__restrict__ seg_offsets, const int32_t *__restrict__ seg_adapter, int64_t S,
     float *__restrict__ part) {
+  // the dependent GEMM grid may launch at once: its weight stream needs
+  // nothing from here, and it waits for this grid to complete before it
+  // reads the partial sums
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int unit = blockIdx.x * (kDecThreads / 32) + warp;  // (token, K slice)
   const int64_t i = unit / kDecKSplit;
@@ -54,23 +59,30 @@ __global__ void __launch_bounds__(kDecThreads) decode_shrink_kernel(
     }
   }
   float *out = part + (i * kDecKSplit + ks) * kDecMaxRank;
-  // K slice of this warp, in 16-element pieces (K % 16 == 0)
+  // K slice of this warp, in 16-element pieces (K % 16 == 0); lane = piece
+  // (lane & 15) of each group of 16 pieces x half (lane >> 4) of each group
+  // of 16 ranks, so that all lanes load at once
   const int64_t pieces = K / 16;
   const int64_t p0 = pieces * ks / kDecKSplit, p1 = pieces * (ks + 1) / kDecKSplit;
+  const int pl = lane & 15, hf = lane >> 4;
+  // the codes and scales come from the quantizer (a no-op unless this grid
+  // is launched as its programmatic dependent)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const float xs = x_scale[i];
-  for (int j0 = 0; j0 < r; j0 += 8) {
+  for (int j0 = 0; j0 < r; j0 += 16) {
+    const int jb = j0 + 8 * hf;  // this lane's 8 ranks (rows up to the padded rank exist)
     float acc[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-    for (int64_t p = p0 + lane; p < p1; p += 32) {
+    for (int64_t p = p0 + pl; p < p1; p += 16) {
       // all loads of this piece first, then the products
       const uint4 xr = __ldg(reinterpret_cast<const uint4 *>(Xq + i * K + p * 16));
       uint4 av[8][2];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const uint16_t *ap = A_pack + static_cast<int64_t>(off + j0 + j) * K + p * 16;
-        av[j][0] = __ldg(reinterpret_cast<const uint4 *>(ap));  // rows up to the padded
-        av[j][1] = __ldg(reinterpret_cast<const uint4 *>(ap + 8));  // rank exist (zeros)
+        const uint16_t *ap = A_pack + static_cast<int64_t>(off + jb + j) * K + p * 16;
+        av[j][0] = __ldg(reinterpret_cast<const uint4 *>(ap));
+        av[j][1] = __ldg(reinterpret_cast<const uint4 *>(ap + 8));
       }
       const uint32_t w4[4] = {xr.x, xr.y, xr.z, xr.w};
       float xv[16];
@@ -90,29 +102,32 @@ __global__ void __launch_bounds__(kDecThreads) decode_shrink_kernel(
         acc[j] += sacc;
       }
     }
+    // sum over the 16 piece lanes of each half, in a fixed order
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       float v = acc[j];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0 && j0 + j < r) out[j0 + j] = xs * v;
+      for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (pl == 0 && jb + j < r) out[jb + j] = xs * v;
     }
   }
-  // the dependent GEMM grid may start once every block got here
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
 // kernel 2: int8 GEMM over 32 output channels, then the LoRA expand.
-// Warp 8 streams this block's 32 rows of Wq through a ring of 128-byte-wide
-// TMA tiles (128-byte swizzle: the 8 rows an MMA fragment load touches sit in
-// distinct banks).  Compute warp w owns tokens [16*(w&3), +16) and channels
-// [16*(w>>2), +16) over the whole K, so no cross-warp reduction is needed.
+// Warp 8 streams this block's 32 rows of Wq and the tokens' Xq through a ring
+// of stages of 256 K-bytes, each two 128-byte-wide TMA tiles per operand
+// (128-byte swizzle: the 8 rows an MMA fragment load touches sit in distinct
+// banks); the four copies of a stage are issued by four lanes in one warp
+// instruction, since one thread's copies are issued one after another.
+// Compute warp w owns tokens [16*(w&3), +16) and channels [16*(w>>2), +16)
+// over the whole K, so no cross-warp reduction is needed.
 // ---------------------------------------------------------------------------
-constexpr int kDecStages = 16;
+constexpr int kDecStages = 8;
+constexpr int kDecKStage = 256;                   // K bytes per stage (two tiles)
 constexpr int kDecWBytes = kDecCols * 128;        // Wq tile: 32 rows x 128 K-bytes
 constexpr int kDecXBytes = kDecMaxM * 128;        // Xq tile: 64 rows x 128 K-bytes
-constexpr int kDecStageBytes = kDecWBytes + kDecXBytes;
+constexpr int kDecStageBytes = 2 * (kDecWBytes + kDecXBytes);
 constexpr int kDecComputeWarps = 8;
 constexpr int kDecGemmThreads = 32 * (kDecComputeWarps + 1);
 
@@ -155,7 +170,7 @@ __global__ void __launch_bounds__(kDecGemmThreads) decode_gemm_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kDecCols;
   const bool lora = (part != nullptr);
-  const int nk = (mode == 2) ? 0 : static_cast<int>((K + 127) / 128);
+  const int nk = (mode == 2) ? 0 : static_cast<int>((K + kDecKStage - 1) / kDecKStage);
   const int kb_first = (nk > 0) ? static_cast<int>((blockIdx.x * 5u) % static_cast<unsigned>(nk)) : 0;
 
   if (threadIdx.x == 0) {
@@ -170,27 +185,48 @@ __global__ void __launch_bounds__(kDecGemmThreads) decode_gemm_kernel(
 
   if (warp == kDecComputeWarps) {
     // ---------------------------------------------------------- producer
-    if (lane == 0) {
-      prefetch_tmap(&tm_w);
-      prefetch_tmap(&tm_x);
+    // lane 0 waits for a free stage and posts its bytes; lanes 0-3 then copy
+    // Wq tile 0, Wq tile 1, Xq tile 0 and Xq tile 1 of the stage together
+    int issued = 0;
+    {
+      if (lane == 0) {
+        prefetch_tmap(&tm_w);
+        prefetch_tmap(&tm_x);
+      }
       uint32_t phase = 0;
-      int st = 0, issued = 0;
+      int st = 0;
+      // blocks start their K walk at different stages so that they do not
+      // all read the same Xq tile (from the same L2 lines) at once
+      int kk = kb_first;
       for (int kb = 0; kb < nk; ++kb) {
-        if (!mbar_wait(&ctl.empty[st], phase ^ 1u, timeout_ns, abort_flag)) {
-          *reinterpret_cast<volatile int *>(abort_flag) = 1;
-          record_device_error(SQ_ERR_DEVICE_TIMEOUT);
+        bool got = true;
+        if (lane == 0) {
+          got = mbar_wait(&ctl.empty[st], phase ^ 1u, timeout_ns, abort_flag);
+          if (got) mbar_arrive_expect_tx(&ctl.full[st], kDecStageBytes);
+        }
+        if (!__shfl_sync(0xffffffffu, got, 0)) {
+          if (lane == 0) {
+            *reinterpret_cast<volatile int *>(abort_flag) = 1;
+            record_device_error(SQ_ERR_DEVICE_TIMEOUT);
+          }
           break;
         }
-        mbar_arrive_expect_tx(&ctl.full[st], kDecStageBytes);
-        // blocks start their K walk at different K blocks so that they do not
-        // all read the same Xq tile (from the same L2 lines) at once
-        const int kk = (kb + kb_first) % nk;
-        tma_load_2d(ring + st * kDecStageBytes, &tm_w, &ctl.full[st], kk * 128,
-                    static_cast<int32_t>(n0));
-        tma_load_2d(ring + st * kDecStageBytes + kDecWBytes, &tm_x, &ctl.full[st], kk * 128, 0);
+        if (lane < 4) {
+          const int tile = lane & 1;  // K half of the stage
+          const int32_t x = kk * kDecKStage + tile * 128;
+          if (lane < 2)
+            tma_load_2d(ring + st * kDecStageBytes + tile * kDecWBytes, &tm_w, &ctl.full[st], x,
+                        static_cast<int32_t>(n0));
+          else
+            tma_load_2d(ring + st * kDecStageBytes + 2 * kDecWBytes + tile * kDecXBytes, &tm_x,
+                        &ctl.full[st], x, 0);
+        }
         ++issued;
+        if (++kk == nk) kk = 0;
         if (++st == kDecStages) { st = 0; phase ^= 1u; }
       }
+    }
+    if (lane == 0) {
       // every issued copy must land before the block exits: wait for the
       // last use of each stage
       volatile int never = 0;
@@ -209,6 +245,23 @@ __global__ void __launch_bounds__(kDecGemmThreads) decode_gemm_kernel(
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[nt][e] = 0;
     const int ra = mt * 16 + g, rb = ra + 8;  // token rows of this lane's A fragments
+    // adapter of each token (warps 0-3 cover the 64 tokens), looked up while
+    // the first stages load; read by all compute warps after the K loop
+    if (lora && nh == 0 && lane < 16) {
+      const int i = mt * 16 + lane;
+      int off = 0, r = 0;
+      if (i < M) {
+        const int a = token_adapter(seg_offsets, seg_adapter, S, n_adapters, i);
+        if (a >= 0) {
+          off = lora_offset[a];
+          r = lora_rank[a];
+          if (off < 0 || (off & 15) || r <= 0 || r > kDecMaxRank || off + ((r + 15) & ~15) > R)
+            r = 0;
+        }
+      }
+      ctl.off[i] = off;
+      ctl.rank[i] = r;
+    }
     uint32_t phase = 0;
     int st = 0;
     bool ok = true;
@@ -216,10 +269,11 @@ __global__ void __launch_bounds__(kDecGemmThreads) decode_gemm_kernel(
       // the warp leaves together: the mma.sync below needs all lanes
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ctl.full[st], phase, timeout_ns, abort_flag))))
         break;
-      const uint8_t *wt = ring + st * kDecStageBytes;
-      const uint8_t *xt = wt + kDecWBytes;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int hh = 0; hh < 4; ++hh) {
+        const int h = hh & 1;  // 64-byte half of a 128-byte tile row
+        const uint8_t *wt = ring + st * kDecStageBytes + (hh >> 1) * kDecWBytes;
+        const uint8_t *xt = ring + st * kDecStageBytes + 2 * kDecWBytes + (hh >> 1) * kDecXBytes;
         // 16 contiguous K bytes (chunk 4h + tig of the 128-byte row, stored
         // 128B-swizzled) of each operand row; the K order inside the 64 bytes
         // is a permutation that A and B share
@@ -247,49 +301,13 @@ __global__ void __launch_bounds__(kDecGemmThreads) decode_gemm_kernel(
       *reinterpret_cast<volatile int *>(abort_flag) = 1;
       record_device_error(SQ_ERR_DEVICE_TIMEOUT);
     }
-    // ---- LoRA intermediate: adapter of each token (warps 0-3 cover the 64
-    //      tokens), then T summed over the shrink's K slices.  Every compute
-    //      warp meets both barriers, also after a wait that ran out.
+    // ---- LoRA: every compute warp has finished reading the ring (T may
+    //      overwrite it) and the adapter table is complete; the B' columns of
+    //      the first 16 ranks are loaded before the shrink's partial sums are
+    //      waited for, then T = sum of the partials over the shrink's K slices.
+    //      Every compute warp meets both barriers, also after a wait that ran out.
     float (*Tm)[kDecMaxRank] = reinterpret_cast<float (*)[kDecMaxRank]>(ring);
-    if (lora) {
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      if (nh == 0 && lane < 16) {
-        const int i = mt * 16 + lane;
-        int off = 0, r = 0;
-        if (i < M) {
-          const int a = token_adapter(seg_offsets, seg_adapter, S, n_adapters, i);
-          if (a >= 0) {
-            off = lora_offset[a];
-            r = lora_rank[a];
-            if (off < 0 || (off & 15) || r <= 0 || r > kDecMaxRank || off + ((r + 15) & ~15) > R)
-              r = 0;
-          }
-        }
-        ctl.off[i] = off;
-        ctl.rank[i] = r;
-      }
-      // every compute warp has finished reading the ring: T may overwrite it
-      asm volatile("bar.sync 1, %0;" ::"r"(32 * kDecComputeWarps) : "memory");
-      // four threads per token, each summing every fourth column; all the
-      // partial loads of a column are independent
-      {
-        const int i = threadIdx.x >> 2, jq = threadIdx.x & 3;
-        const int r = (i < M) ? ctl.rank[i] : 0;
-        const int rpad = (r + 15) & ~15;
-        for (int j = jq; j < rpad; j += 4) {
-          float t = 0.f;  // zero in the padding columns (the expand reads them)
-          if (j < r) {
-            float pv[kDecKSplit];
-#pragma unroll
-            for (int ks = 0; ks < kDecKSplit; ++ks) pv[ks] = part[(i * kDecKSplit + ks) * kDecMaxRank + j];
-#pragma unroll
-            for (int ks = 0; ks < kDecKSplit; ++ks) t += pv[ks];
-          }
-          Tm[i][j] = t;
-        }
-      }
-      asm volatile("bar.sync 1, %0;" ::"r"(32 * kDecComputeWarps) : "memory");
-    }
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * kDecComputeWarps) : "memory");
     // lane: rows ra, rb; channels n0 + 16nh + 8nt + 2tig + {0,1}
     float d[2][2][2];  // [half][nt][channel of the pair]
     int rr[2], oo[2];
@@ -302,9 +320,7 @@ __global__ void __launch_bounds__(kDecGemmThreads) decode_gemm_kernel(
       for (int nt = 0; nt < 2; ++nt) d[half][nt][0] = d[half][nt][1] = 0.f;
     }
     const int rmax = max(rr[0], rr[1]);
-    for (int j0 = 0; j0 < rmax; j0 += 8) {
-      // issue every B' load of this column group before using any
-      uint4 bv[2][2][2];  // [half][nt][channel]
+    auto load_b = [&](int j0, uint4 (&bv)[2][2][2]) {
 #pragma unroll
       for (int half = 0; half < 2; ++half)
 #pragma unroll
@@ -316,6 +332,55 @@ __global__ void __launch_bounds__(kDecGemmThreads) decode_gemm_kernel(
                                   ? __ldg(reinterpret_cast<const uint4 *>(B_pack + (n + c) * R + oo[half] + j0))
                                   : make_uint4(0, 0, 0, 0);
         }
+    };
+    uint4 bpre[2][2][2][2];  // column groups 0 and 1 (ranks 0-15), loaded early
+    load_b(0, bpre[0]);
+    load_b(8, bpre[1]);
+    if (lora) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      // four threads per token, each summing every fourth column; the 16
+      // partials of four columns are loaded before any is added
+      const int i = threadIdx.x >> 2, jq = threadIdx.x & 3;
+      const int r = (i < M) ? ctl.rank[i] : 0;
+      const int rpad = (r + 15) & ~15;
+      for (int jb = 0; jb < rpad; jb += 16) {
+        float pv[4][kDecKSplit];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int j = jb + jq + 4 * m;
+#pragma unroll
+          for (int ks = 0; ks < kDecKSplit; ++ks)
+            pv[m][ks] = (j < r) ? part[(i * kDecKSplit + ks) * kDecMaxRank + j] : 0.f;
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          float t = 0.f;  // zero in the padding columns (the expand reads them)
+#pragma unroll
+          for (int ks = 0; ks < kDecKSplit; ++ks) t += pv[m][ks];
+          Tm[i][jb + jq + 4 * m] = t;
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(32 * kDecComputeWarps) : "memory");
+    }
+    for (int j0 = 0; j0 < rmax; j0 += 8) {
+      uint4 bv[2][2][2];  // [half][nt][channel]
+      if (j0 == 0) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half)
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) bv[half][nt][c] = bpre[0][half][nt][c];
+      } else if (j0 == 8) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half)
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) bv[half][nt][c] = bpre[1][half][nt][c];
+      } else {
+        load_b(j0, bv);
+      }
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         if (j0 >= rr[half]) continue;
