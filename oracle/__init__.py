@@ -61,6 +61,8 @@ def lib():
             "sqo_token_adapter": ([P, P, I64, I32, I64], I32),
             "sqo_linear_lora_rows": ([P, P, P, P, I64, I64, I64, I32, P, P, P, P, P, I64,
                                       P, I64, P, P, P], None),
+            "sqo_linear_lora_raw_rows": ([P, P, P, P, P, I64, I64, I64, I32, P, P, P, P, P,
+                                          I64, P, I64, P, P], None),
             "sqo_reference_rows": ([P, I32, P, I64, I64, I64, I32, P, P, P, P, P, P, I64,
                                     P, I64, P], None),
             "sqo_smoothed_product_rows": ([P, I32, P, P, I64, I64, P, I64, P], None),
@@ -146,11 +148,12 @@ def quant_act(X: np.ndarray, s: np.ndarray):
     return Xq, xs
 
 
-def prepare_lora(A: np.ndarray, B: np.ndarray, s: np.ndarray, lora_alpha: float):
-    """A_s = bf16(A*s) along K, B_s = bf16(B*lora_alpha/r). Returns bf16 bits."""
+def prepare_lora(A: np.ndarray, B: np.ndarray, s: Optional[np.ndarray], lora_alpha: float):
+    """A_s = bf16(A*s) along K (A unchanged when s is None: the raw-input
+    reading), B_s = bf16(B*lora_alpha/r). Returns bf16 bits."""
     A = _c(A, np.uint16)
     B = _c(B, np.uint16)
-    s = _c(s, np.float32)
+    s = None if s is None else _c(s, np.float32)
     r, K = A.shape
     N = B.shape[0]
     assert B.shape == (N, r)
@@ -224,6 +227,39 @@ def linear_lora_rows(Xq, x_scale, Wq, w_scale, A_s: List[np.ndarray], B_s: List[
                                _ptr_array(A_s), _ptr_array(B_s), _p(ranks), _p(so), _p(sa),
                                sa.shape[0], _p(rows), R, _p(Y), _p(D), _p(A))
     for k, v in (("Y", Y), ("delta", D), ("acc", A)):
+        if v is not None:
+            out[k] = v
+    return out
+
+
+def linear_lora_raw_rows(X, Xq, x_scale, Wq, w_scale, A: List[np.ndarray], B_s: List[np.ndarray],
+                         seg_offsets, seg_adapter, rows: Optional[Sequence[int]] = None,
+                         want=("Y", "delta")):
+    """Raw-input reading of the LoRA path (fp64): T = X A^T from the bf16
+    activations and the adapters as given, delta = T B_s^T, Y = dequantized
+    W8A8 output + delta, for the selected tokens.  X must be bf16 bits."""
+    X = _c(X, np.uint16)
+    Xq = _c(Xq, np.int8)
+    Wq = _c(Wq, np.int8)
+    xs = _c(x_scale, np.float32)
+    ws = _c(w_scale, np.float32)
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    assert X.shape == (M, K)
+    A = [_c(a, np.uint16) for a in A]
+    B_s = [_c(b, np.uint16) for b in B_s]
+    ranks = np.array([a.shape[0] for a in A] or [0], np.int64)
+    so = _c(seg_offsets, np.int32)
+    sa = _c(seg_adapter, np.int32)
+    rows = np.arange(M, dtype=np.int64) if rows is None else _c(rows, np.int64)
+    R = rows.shape[0]
+    Y = np.zeros((R, N), np.float64) if "Y" in want else None
+    D = np.zeros((R, N), np.float64) if "delta" in want else None
+    lib().sqo_linear_lora_raw_rows(_p(X), _p(Xq), _p(xs), _p(Wq), _p(ws), M, N, K, len(A),
+                                   _ptr_array(A), _ptr_array(B_s), _p(ranks), _p(so), _p(sa),
+                                   sa.shape[0], _p(rows), R, _p(Y), _p(D))
+    out = {}
+    for k, v in (("Y", Y), ("delta", D)):
         if v is not None:
             out[k] = v
     return out

@@ -197,9 +197,11 @@ void sqo_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s,
                       int64_t r, int64_t K, int64_t N, float lora_alpha,
                       uint16_t *A_s, uint16_t *B_s) {
   float scale = rn32((double)lora_alpha / (double)r);
+  /* s == NULL: the raw-input reading, A is kept as given (no smoothing fold) */
   for (int64_t j = 0; j < r; ++j)
     for (int64_t k = 0; k < K; ++k)
-      A_s[j * K + k] = rn_bf16(rn32(bf16_value(A[j * K + k]) * (double)s[k]));
+      A_s[j * K + k] = s ? rn_bf16(rn32(bf16_value(A[j * K + k]) * (double)s[k]))
+                         : A[j * K + k];
   for (int64_t n = 0; n < N; ++n)
     for (int64_t j = 0; j < r; ++j)
       B_s[n * r + j] = rn_bf16(rn32(bf16_value(B[n * r + j]) * (double)scale));
@@ -288,6 +290,52 @@ void sqo_linear_lora_rows(const int8_t *Xq, const float *x_scale, const int8_t *
       if (acc) acc[t * N + n] = sum;
       if (delta) delta[t * N + n] = d;
       if (Y) Y[t * N + n] = base + d;
+    }
+    free(T);
+  }
+}
+
+/* ---- [IS] Pitch, raw-input reading: the LoRA path in BF16 on the layer's
+ * own (unquantized) activations, added to the dequantized INT8 output -----
+ *   base[i,n]  = acc[i,n] * x_scale_i * w_scale_n           (as above)
+ *   T[i,j]     = sum_k X[i,k] * A[a][j,k]                   (X bf16, A as given)
+ *   delta[i,n] = sum_j T[i,j] * B_s[a][n,j]
+ *   Y[i,n]     = base[i,n] + delta[i,n]
+ * all in fp64.  X must be bf16 (dtype SQO_BF16).  Any of Y / delta may be NULL. */
+void sqo_linear_lora_raw_rows(const uint16_t *X, const int8_t *Xq, const float *x_scale,
+                              const int8_t *Wq, const float *w_scale, int64_t M, int64_t N,
+                              int64_t K, int n_adapters, const uint16_t *const *A,
+                              const uint16_t *const *B_s, const int64_t *ranks,
+                              const int32_t *seg_offsets, const int32_t *seg_adapter,
+                              int64_t S, const int64_t *rows, int64_t nrows, double *Y,
+                              double *delta) {
+  (void)M;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t t = 0; t < nrows; ++t) {
+    int64_t i = rows[t];
+    int a = sqo_token_adapter(seg_offsets, seg_adapter, S, n_adapters, i);
+    double xs = (double)x_scale[i];
+    double *T = NULL;
+    int64_t r = 0;
+    if (a >= 0) {
+      r = ranks[a];
+      T = (double *)calloc((size_t)(r > 0 ? r : 1), sizeof(double));
+      for (int64_t j = 0; j < r; ++j) {
+        double sum = 0.0;
+        for (int64_t k = 0; k < K; ++k)
+          sum += bf16_value(X[i * K + k]) * bf16_value(A[a][j * K + k]);
+        T[j] = sum;
+      }
+    }
+    for (int64_t n = 0; n < N; ++n) {
+      double d = 0.0;
+      for (int64_t j = 0; j < r; ++j) d += T[j] * bf16_value(B_s[a][n * r + j]);
+      if (delta) delta[t * N + n] = d;
+      if (Y) {
+        int64_t sum = 0;
+        for (int64_t k = 0; k < K; ++k) sum += (int64_t)Xq[i * K + k] * (int64_t)Wq[n * K + k];
+        Y[t * N + n] = (double)sum * xs * (double)w_scale[n] + d;
+      }
     }
     free(T);
   }

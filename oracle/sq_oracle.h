@@ -46,6 +46,13 @@ void sqo_linear_lora_rows(const int8_t *Xq, const float *x_scale, const int8_t *
                           const int32_t *seg_offsets, const int32_t *seg_adapter, int64_t S,
                           const int64_t *rows, int64_t nrows, double *Y, double *delta,
                           int64_t *acc);
+void sqo_linear_lora_raw_rows(const uint16_t *X, const int8_t *Xq, const float *x_scale,
+                              const int8_t *Wq, const float *w_scale, int64_t M, int64_t N,
+                              int64_t K, int n_adapters, const uint16_t *const *A,
+                              const uint16_t *const *B_s, const int64_t *ranks,
+                              const int32_t *seg_offsets, const int32_t *seg_adapter,
+                              int64_t S, const int64_t *rows, int64_t nrows, double *Y,
+                              double *delta);
 void sqo_reference_rows(const void *X, int dtype, const uint16_t *W, int64_t M, int64_t N,
                         int64_t K, int n_adapters, const uint16_t *const *A,
                         const uint16_t *const *B, const int64_t *ranks,
