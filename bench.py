@@ -53,6 +53,9 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wk.SPECS))
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--lora-input", choices=["dequant", "raw"], default="dequant",
+                   help="what the LoRA path reads: the dequantized codes (default) or the "
+                        "raw bf16 activations (sq_lora_shrink_raw + sq_linear_lora_from_t)")
     return p.parse_args()
 
 
@@ -187,28 +190,33 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # CPU oracle (reported baseline; test infrastructure, timed as it stands)
 # ---------------------------------------------------------------------------
-def oracle_step(P, wl, rows):
+def oracle_step(P, wl, rows, raw=False):
     import oracle
     Xq, xs = oracle.quant_act(wl.X[rows], P.s)
     ad = wk.row_adapter(wl.seg_offsets, wl.seg_adapter, wl.M, len(wl.adapters))
     # the sampled tokens keep their own adapters: one segment per token
     so = np.arange(len(rows) + 1, dtype=np.int32)
     sa = ad[rows].astype(np.int32)
-    oracle.linear_lora_rows(Xq, xs, P.Wq, P.w_scale, P.A_s, P.B_s, so, sa, want=("Y",))
+    if raw:
+        oracle.linear_lora_raw_rows(wl.X[rows], Xq, xs, P.Wq, P.w_scale, [a.A for a in wl.adapters],
+                                    P.B_s, so, sa, want=("Y",))
+    else:
+        oracle.linear_lora_rows(Xq, xs, P.Wq, P.w_scale, P.A_s, P.B_s, so, sa, want=("Y",))
 
 
-def cpu_baseline(wl, sample_rows=None):
+def cpu_baseline(wl, sample_rows=None, raw=False):
     import oracle
     P = oracle.Prepared(wl)
     rows = np.arange(wl.M if sample_rows is None else min(sample_rows, wl.M))
     t0 = time.perf_counter()
-    oracle_step(P, wl, rows)
+    oracle_step(P, wl, rows, raw)
     dt = time.perf_counter() - t0
     ops = 2 * len(rows) * wl.N * wl.K
     return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": oracle.num_threads(),
             "kind": "oracle",
             "sample": f"{len(rows)} of {wl.M} tokens, whole hot path (quantize, int64 GEMM, fp64 "
-                      f"dequant + LoRA), one pass, {dt:.2f} s",
+                      f"dequant + LoRA on the {'raw activations' if raw else 'dequantized codes'}), "
+                      f"one pass, {dt:.2f} s",
             "tokens_per_s": len(rows) / dt}
 
 
@@ -225,7 +233,7 @@ def run_reference(args):
     for i in range(args.warmup + args.steps):
         rows = np.sort(rng.choice(wl.M, size=sample, replace=False))
         t0 = time.perf_counter()
-        oracle_step(P, wl, rows)
+        oracle_step(P, wl, rows, args.lora_input == "raw")
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             times.append(dt)
@@ -273,7 +281,7 @@ def run_ours(args):
     wl = wk.make_workload(args.workload)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl)
+        cpu = cpu_baseline(wl, raw=args.lora_input == "raw")
 
     M, K, N = wl.M, wl.K, wl.N
 
@@ -296,14 +304,18 @@ def run_ours(args):
     w_scale = torch.empty(N, dtype=torch.float32, device=dev)
     sq.sq_quantize_weight(W, s, Wq, w_scale)
     del W
+    raw = args.lora_input == "raw"
+    if raw and not wl.x_is_bf16:
+        raise SystemExit("--lora-input raw needs bf16 activations")
     lora = sq.LoraPack.build([h2d(a.A) for a in wl.adapters], [h2d(a.B) for a in wl.adapters],
-                             [a.lora_alpha for a in wl.adapters], s)
+                             [a.lora_alpha for a in wl.adapters], None if raw else s)
     seg_offsets = h2d(wl.seg_offsets)
     seg_adapter = h2d(wl.seg_adapter)
     Xq = torch.empty((M, K), dtype=torch.int8, device=dev)
     x_scale = torch.empty(M, dtype=torch.float32, device=dev)
-    ws = torch.empty(max(sq.sq_linear_lora_workspace_size(M, lora.R), 256), dtype=torch.uint8,
-                     device=dev)
+    ws_bytes = (sq.sq_lora_t_workspace_size(M, lora.R) if raw
+                else sq.sq_linear_lora_workspace_size(M, lora.R))
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     flush_read = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
@@ -316,7 +328,11 @@ def run_ours(args):
 
     def step():
         sq.sq_quant_act(X, s, Xq, x_scale)
-        sq.sq_linear_lora(Xq, x_scale, Wq, w_scale, lora, seg_offsets, seg_adapter, Y, ws)
+        if raw:
+            sq.sq_lora_shrink_raw(X, lora, seg_offsets, seg_adapter, ws)
+            sq.sq_linear_lora_from_t(Xq, x_scale, Wq, w_scale, lora, Y, ws)
+        else:
+            sq.sq_linear_lora(Xq, x_scale, Wq, w_scale, lora, seg_offsets, seg_adapter, Y, ws)
 
     launches_per_step = 3  # quantize, LoRA shrink, fused GEMM
 
@@ -389,7 +405,7 @@ def run_ours(args):
     gemm_tops = ops_step / gemm_avg_s / 1e12
     peaks, peak_kind = measured_peaks()
     int8_peak = 2.0 * float(peaks["bf16_tflops"])  # dense int8 = 2x dense bf16 (nominal ratio)
-    if M <= DECODE_MAX_M:
+    if M <= DECODE_MAX_M and not raw:
         # decode form: bound by streaming Wq and the adapters from HBM; the
         # timed region is the whole layer call (shrink + GEMM kernels)
         nbytes = decode_layer_bytes(wl)
@@ -424,7 +440,9 @@ def run_ours(args):
         "config": {"workload": wl.spec.name, "M": M, "K": K, "N": N,
                    "adapters": len(wl.adapters), "ranks": sorted(set(a.r for a in wl.adapters)),
                    "segments": int(len(wl.seg_adapter)), "alpha": wl.alpha,
-                   "step": "sq_quant_act + sq_linear_lora (shrink + fused GEMM)",
+                   "step": ("sq_quant_act + sq_lora_shrink_raw + sq_linear_lora_from_t "
+                            "(LoRA on the raw bf16 activations)" if raw else
+                            "sq_quant_act + sq_linear_lora (shrink + fused GEMM)"),
                    "l2": "flushed between timed steps (256 MiB write + 256 MiB read, untimed)",
                    "parallelism": f"replicas x{world}"},
         "tokens_per_s": tok_s,

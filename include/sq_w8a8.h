@@ -98,9 +98,10 @@ int sq_set_wait_timeout_ns(uint64_t ns);
  * status. */
 int sq_selftest_wait_timeout(uint64_t timeout_ns, void *stream);
 
-/* Measurement aid: when both are non-NULL, sq_linear_lora records the
- * cudaEvent_t `before` on its stream right before it launches the fused GEMM
- * kernel and `after` right after, so a caller can time that kernel alone.
+/* Measurement aid: when both are non-NULL, sq_linear_lora (and
+ * sq_linear_lora_from_t) records the cudaEvent_t `before` on its stream right
+ * before it launches the fused GEMM kernel and `after` right after, so a
+ * caller can time that kernel alone.
  * NULL disables.  Host-side setting for later calls. */
 int sq_set_gemm_events(void *before, void *after);
 
@@ -142,7 +143,8 @@ int sq_quantize_weight(const uint16_t *W, const float *s, int64_t N, int64_t K,
  * and still compute X*A^T; folding lora_alpha/r into B applies the LoRA
  * scaling once, offline.  This call writes adapter (A [r,K], B [N,r], both
  * bf16, 1 <= r <= SQ_MAX_LORA_RANK) at column offset `off` (a multiple of 16)
- * of a pack of width R. */
+ * of a pack of width R.  s == NULL packs A unchanged (the raw-input reading,
+ * see sq_lora_shrink_raw). */
 int sq_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s, int64_t r,
                     int64_t K, int64_t N, float lora_alpha, int64_t R, int64_t off,
                     uint16_t *A_pack, uint16_t *B_pack, void *stream);
@@ -224,6 +226,48 @@ int sq_lora_delta(const int8_t *Xq, const float *x_scale, int64_t M, int64_t N,
                   int64_t R, const int32_t *seg_offsets, const int32_t *seg_adapter,
                   int64_t S, float *delta, void *workspace, size_t workspace_bytes,
                   void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Raw-input reading of the LoRA path ("[Feature]: LoRA support for W8A8
+ * SmoothQuant", Pitch: the low-rank path runs in BF16 after the INT8 GEMM
+ * and is added to the dequantized output), taken on the layer's own bf16
+ * activations instead of the dequantized codes:
+ *   T[i,j] = sum_k X[i,k] * A_a[j,k]      (X bf16, A_a the adapter as given)
+ *   Y[i,n] = bf16( f32(acc[i,n]) * x_scale_i * w_scale_n + sum_j T[i,j] * B_pack[n, off_a+j] )
+ * The adapters are packed by sq_prepare_lora with s == NULL (A unchanged,
+ * B scaled by lora_alpha/r as above).  T is kept in a caller-provided
+ * workspace between the two calls.
+ * ------------------------------------------------------------------------ */
+
+/* Bytes of workspace for the T planes and mask words of M tokens and a pack
+ * of width R (any M; 0 when R == 0 or M == 0). */
+size_t sq_lora_t_workspace_size(int64_t M, int64_t R);
+
+/* T for every token, written to `workspace` (>= sq_lora_t_workspace_size(M, R)
+ * bytes, 256-byte aligned, device memory; contents replaced).  X [M,K] bf16
+ * device; A_pack [R,K] bf16 packed with s == NULL; lora_offset, lora_rank,
+ * seg_offsets, seg_adapter as for sq_linear_lora (tokens without an adapter
+ * get T = 0).  Errors: SQ_ERR_INVALID_ARG (null or misaligned pointers),
+ * SQ_ERR_UNSUPPORTED_SHAPE (K % 16, R % 16, limits), SQ_ERR_WORKSPACE. */
+int sq_lora_shrink_raw(const uint16_t *X, int64_t M, int64_t K, const uint16_t *A_pack,
+                       const int32_t *lora_offset, const int32_t *lora_rank, int n_adapters,
+                       int64_t R, const int32_t *seg_offsets, const int32_t *seg_adapter,
+                       int64_t S, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Y [M,N] bf16 = dequantized W8A8 output + T B_pack^T, with T from
+ * sq_lora_shrink_raw on the same workspace, M and R (R == 0: plain W8A8).
+ * Xq, x_scale, Wq, w_scale as for sq_linear_lora; the fused tensor-core GEMM
+ * for every M.  Errors as sq_linear_lora. */
+int sq_linear_lora_from_t(const int8_t *Xq, const float *x_scale, const int8_t *Wq,
+                          const float *w_scale, int64_t M, int64_t N, int64_t K,
+                          const uint16_t *B_pack, int64_t R, uint16_t *Y, const void *workspace,
+                          size_t workspace_bytes, void *stream);
+
+/* Test entry: delta [M,N] f32 = T B_pack^T alone, as sq_linear_lora_from_t
+ * adds it (Xq and K only shape the call). */
+int sq_lora_delta_from_t(const int8_t *Xq, int64_t M, int64_t N, int64_t K,
+                         const uint16_t *B_pack, int64_t R, float *delta, const void *workspace,
+                         size_t workspace_bytes, void *stream);
 
 #ifdef __cplusplus
 }

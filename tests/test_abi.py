@@ -107,3 +107,39 @@ def test_offline_validation(lib):
     assert lib.sq_set_wait_timeout_ns(0) == INVALID
     code = ctypes.c_int(0)
     assert lib.sq_get_device_error(None, 0) == INVALID
+
+
+def test_raw_lora_entry_validation(lib):
+    # raw-input reading of the LoRA path: T from bf16 activations, then Y
+    assert lib.sq_lora_t_workspace_size(0, 16) == 0
+    assert lib.sq_lora_t_workspace_size(64, 0) == 0
+    tws = lib.sq_lora_t_workspace_size(64, 32)   # any M: no decode special case
+    assert tws >= 2 * 64 * 32 * 2 + 4 * 8 and tws % 256 == 0
+    f = lib.sq_lora_shrink_raw
+    good = (A, 64, 1024, A, A, A, 2, 32, A, A, 3, A, tws, None)
+
+    def shrink(**kw):
+        names = ("X", "M", "K", "Ap", "off", "rk", "nad", "R", "so", "sa", "S", "w", "wb", "st")
+        a = dict(zip(names, good), **kw)
+        return f(*[a[n] for n in names])
+
+    assert shrink(K=1000) == SHAPE
+    assert shrink(R=24) == SHAPE
+    assert shrink(R=0) == INVALID
+    assert shrink(wb=tws - 1) == WORKSPACE
+    assert shrink(w=A + 16) == WORKSPACE
+    assert shrink(X=A + 2) == INVALID
+    assert shrink(off=None) == INVALID
+    assert shrink() in (CUDA, DEVICE)
+    g = lib.sq_linear_lora_from_t
+    assert g(A, A, A, A, 64, 100, 1024, A, 32, A, A, tws, None) == SHAPE      # N % 16
+    assert g(A, A, A, A, 64, 128, 1024, A, 24, A, A, tws, None) == SHAPE      # R % 16
+    assert g(A, A, A, A, 64, 128, 1024, None, 32, A, A, tws, None) == INVALID  # B_pack
+    assert g(A, A, A, A, 64, 128, 1024, A, 32, A, A, tws - 1, None) == WORKSPACE
+    assert g(A, A, A, A, 64, 128, 1024, A, 32, A, A, tws, None) in (CUDA, DEVICE)
+    assert g(A, A, A, A, 64, 128, 1024, None, 0, A, None, 0, None) in (CUDA, DEVICE)  # plain W8A8
+    h = lib.sq_lora_delta_from_t
+    assert h(A, 64, 128, 1024, A, 32, A + 4, A, tws, None) == INVALID        # delta alignment
+    assert h(A, 64, 128, 1024, A, 32, A, A, tws, None) in (CUDA, DEVICE)
+    # s == NULL is the raw-input packing (A unchanged), not an argument error
+    assert lib.sq_prepare_lora(A, A, None, 8, 64, 32, 16.0, 16, 0, A, A, None) in (CUDA, DEVICE)

@@ -22,7 +22,8 @@ __all__ = [
     "sq_get_device_error", "sq_set_wait_timeout_ns", "sq_set_gemm_events", "sq_selftest_wait_timeout", "sq_act_absmax_update", "sq_weight_absmax",
     "sq_compute_smoothing", "sq_quantize_weight", "sq_prepare_lora", "sq_quant_act",
     "sq_linear_lora_workspace_size", "sq_linear_lora", "sq_linear_lora_noalloc", "sq_gemm_i32",
-    "sq_lora_delta",
+    "sq_lora_delta", "sq_lora_t_workspace_size", "sq_lora_shrink_raw", "sq_linear_lora_from_t",
+    "sq_lora_delta_from_t",
 ]
 
 SQ_DTYPE_F32 = 0
@@ -166,13 +167,16 @@ class LoraPack:
 
     @classmethod
     def build(cls, As: List, Bs: List, lora_alphas: Sequence[float], s, stream=None) -> "LoraPack":
-        """Pack adapters (A [r,K], B [N,r] bf16 device tensors) with sq_prepare_lora."""
+        """Pack adapters (A [r,K], B [N,r] bf16 device tensors) with sq_prepare_lora.
+
+        s=None packs A unchanged, for the raw-input entry points
+        (sq_lora_shrink_raw / sq_linear_lora_from_t)."""
         import torch
-        K = s.shape[0]
+        K = s.shape[0] if s is not None else As[0].shape[1]
         N = Bs[0].shape[0] if Bs else 0
         ranks = [a.shape[0] for a in As]
         offs, R = cls.layout(ranks)
-        dev = s.device
+        dev = s.device if s is not None else As[0].device
         A_pack = torch.empty((max(R, 1), K), dtype=torch.bfloat16, device=dev)
         B_pack = torch.empty((max(N, 1), max(R, 1)), dtype=torch.bfloat16, device=dev)
         for A, B, la, off in zip(As, Bs, lora_alphas, offs):
@@ -225,6 +229,44 @@ def sq_gemm_i32(Xq, Wq, acc, stream=None) -> None:
     M, K = Xq.shape
     N = Wq.shape[0]
     _check(_lib().sq_gemm_i32(_ptr(Xq), _ptr(Wq), M, N, K, _ptr(acc), _stream(stream)), "sq_gemm_i32")
+
+
+def sq_lora_t_workspace_size(M: int, R: int) -> int:
+    return int(_lib().sq_lora_t_workspace_size(M, R))
+
+
+def sq_lora_shrink_raw(X, lora: LoraPack, seg_offsets, seg_adapter, workspace, stream=None) -> None:
+    """T = X A^T (raw bf16 activations, adapters packed with s=None) into `workspace`."""
+    M, K = X.shape
+    S = 0 if seg_adapter is None else seg_adapter.shape[0]
+    wp, wb = _ws(workspace)
+    _check(_lib().sq_lora_shrink_raw(_ptr(X), M, K, _ptr(lora.A_pack), _ptr(lora.offset),
+                                     _ptr(lora.rank), lora.n_adapters, lora.R, _ptr(seg_offsets),
+                                     _ptr(seg_adapter), S, wp, wb, _stream(stream)),
+           "sq_lora_shrink_raw")
+
+
+def sq_linear_lora_from_t(Xq, x_scale, Wq, w_scale, lora: Optional[LoraPack], Y, workspace,
+                          stream=None) -> None:
+    """Y = dequantized W8A8 output + T B_pack^T with T from sq_lora_shrink_raw."""
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    R = 0 if lora is None else lora.R
+    B = None if lora is None else lora.B_pack
+    wp, wb = _ws(workspace)
+    _check(_lib().sq_linear_lora_from_t(_ptr(Xq), _ptr(x_scale), _ptr(Wq), _ptr(w_scale), M, N, K,
+                                        _ptr(B), R, _ptr(Y), wp, wb, _stream(stream)),
+           "sq_linear_lora_from_t")
+
+
+def sq_lora_delta_from_t(Xq, N: int, lora: Optional[LoraPack], delta, workspace,
+                         stream=None) -> None:
+    M, K = Xq.shape
+    R = 0 if lora is None else lora.R
+    B = None if lora is None else lora.B_pack
+    wp, wb = _ws(workspace)
+    _check(_lib().sq_lora_delta_from_t(_ptr(Xq), M, N, K, _ptr(B), R, _ptr(delta), wp, wb,
+                                       _stream(stream)), "sq_lora_delta_from_t")
 
 
 def sq_lora_delta(Xq, x_scale, N: int, lora: Optional[LoraPack], seg_offsets, seg_adapter, delta,

@@ -58,6 +58,13 @@ static size_t workspace_bytes(int64_t M, int64_t R) {
   return 2 * plane + align256(static_cast<size_t>((M + 15) / 16) * 8);
 }
 
+// T planes and mask words alone (the raw-input entry points, any M)
+static size_t t_workspace_bytes(int64_t M, int64_t R) {
+  if (R <= 0 || M <= 0) return 0;
+  const size_t plane = align256(static_cast<size_t>(M) * static_cast<size_t>(R) * 2);
+  return 2 * plane + align256(static_cast<size_t>((M + 15) / 16) * 8);
+}
+
 static Workspace carve(void *ws, int64_t M, int64_t R) {
   const size_t plane = align256(static_cast<size_t>(M) * static_cast<size_t>(R) * 2);
   uint8_t *p = static_cast<uint8_t *>(ws);
@@ -218,7 +225,9 @@ int sq_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s, int64_
     return SQ_ERR_UNSUPPORTED_SHAPE;
   const int64_t rpad = (r + 15) / 16 * 16;
   if (off + rpad > R) return SQ_ERR_INVALID_ARG;
-  if (!A || !B || !ptr_ok(s) || !ptr_ok(A_pack) || !ptr_ok(B_pack)) return SQ_ERR_INVALID_ARG;
+  // s == NULL packs A as given (raw-input reading of the LoRA path)
+  if (!A || !B || (s && !ptr_ok(s)) || !ptr_ok(A_pack) || !ptr_ok(B_pack))
+    return SQ_ERR_INVALID_ARG;
   int st = check_device();
   if (st) return st;
   const float scale = lora_alpha / static_cast<float>(r);  // IEEE fp32 division
@@ -322,6 +331,89 @@ int sq_lora_delta(const int8_t *Xq, const float *x_scale, int64_t M, int64_t N, 
                   size_t workspace_size, void *stream) {
   return linear_common(Xq, x_scale, nullptr, nullptr, M, N, K, A_pack, B_pack, lora_offset,
                        lora_rank, n_adapters, R, seg_offsets, seg_adapter, S, 2, delta, workspace,
+                       workspace_size, stream);
+}
+
+// ---- raw-input reading of the LoRA path ------------------------------------
+size_t sq_lora_t_workspace_size(int64_t M, int64_t R) { return t_workspace_bytes(M, R); }
+
+int sq_lora_shrink_raw(const uint16_t *X, int64_t M, int64_t K, const uint16_t *A_pack,
+                       const int32_t *lora_offset, const int32_t *lora_rank, int n_adapters,
+                       int64_t R, const int32_t *seg_offsets, const int32_t *seg_adapter,
+                       int64_t S, void *workspace, size_t workspace_size, void *stream) {
+  int st = check_mk(M, K);
+  if (st) return st;
+  if (n_adapters < 0 || R <= 0 || S < 0) return SQ_ERR_INVALID_ARG;
+  if (R % 16 != 0 || R > SQ_MAX_LORA_COLS) return SQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return check_device();
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_size < t_workspace_bytes(M, R))
+    return SQ_ERR_WORKSPACE;
+  if (K > 0 && (!ptr_ok(X) || !ptr_ok(A_pack))) return SQ_ERR_INVALID_ARG;
+  if (n_adapters > 0 && (!lora_offset || !lora_rank)) return SQ_ERR_INVALID_ARG;
+  if (S > 0 && (!seg_offsets || !seg_adapter)) return SQ_ERR_INVALID_ARG;
+  if ((st = check_device())) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Workspace w = carve(workspace, M, R);
+  if (K == 0 || n_adapters == 0 || S == 0)  // no adapter rows or no contraction: T = 0, masks 0
+    return cuda_status(cudaMemsetAsync(workspace, 0, t_workspace_bytes(M, R), s));
+  return cuda_status(launch_lora_shrink_raw(X, M, K, A_pack, lora_offset, lora_rank, n_adapters,
+                                            R, seg_offsets, seg_adapter, S, w.T_hi, w.T_lo, w.mask,
+                                            s));
+}
+
+// Y or the delta alone (mode 0 / 2) from the T planes in the workspace
+static int from_t_common(const int8_t *Xq, const float *x_scale, const int8_t *Wq,
+                         const float *w_scale, int64_t M, int64_t N, int64_t K,
+                         const uint16_t *B_pack, int64_t R, int mode, void *out,
+                         const void *workspace, size_t workspace_size, void *stream) {
+  int st = check_mk(M, K);
+  if (st) return st;
+  if (N < 0 || R < 0) return SQ_ERR_INVALID_ARG;
+  if (N % 16 != 0) return SQ_ERR_UNSUPPORTED_SHAPE;
+  if (R % 16 != 0 || R > SQ_MAX_LORA_COLS) return SQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return check_device();
+  if (!ptr_ok(out)) return SQ_ERR_INVALID_ARG;
+  if (K > 0 && (!ptr_ok(Xq) || (mode == 0 && (!ptr_ok(Wq) || !ptr_ok(x_scale) || !ptr_ok(w_scale)))))
+    return SQ_ERR_INVALID_ARG;
+  const bool lora = R > 0;
+  if (lora && !ptr_ok(B_pack)) return SQ_ERR_INVALID_ARG;
+  if (lora && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+               workspace_size < t_workspace_bytes(M, R)))
+    return SQ_ERR_WORKSPACE;
+  if ((st = check_device())) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t esize = (mode == 0) ? 2 : 4;
+  // K == 0: no contraction and T = 0 (sq_lora_shrink_raw), so the output is 0
+  if (K == 0 || (mode == 2 && !lora))
+    return cuda_status(cudaMemsetAsync(out, 0, static_cast<size_t>(M) * N * esize, s));
+  LoraOperands lo;
+  LoraOperands *lop = nullptr;
+  if (lora) {
+    Workspace w = carve(const_cast<void *>(workspace), M, R);
+    lo = LoraOperands{w.T_hi, w.T_lo, B_pack, w.mask, R};
+    lop = &lo;
+  }
+  const bool timed = (mode == 0) && g_gemm_ev_before != nullptr;
+  if (timed && cudaEventRecord(g_gemm_ev_before, s) != cudaSuccess) return SQ_ERR_CUDA;
+  cudaError_t e = launch_w8a8_gemm(Xq, Wq, x_scale, w_scale, M, N, K, mode, out, lop, s);
+  if (e != cudaSuccess) return SQ_ERR_CUDA;
+  if (timed && cudaEventRecord(g_gemm_ev_after, s) != cudaSuccess) return SQ_ERR_CUDA;
+  return SQ_OK;
+}
+
+int sq_linear_lora_from_t(const int8_t *Xq, const float *x_scale, const int8_t *Wq,
+                          const float *w_scale, int64_t M, int64_t N, int64_t K,
+                          const uint16_t *B_pack, int64_t R, uint16_t *Y, const void *workspace,
+                          size_t workspace_size, void *stream) {
+  return from_t_common(Xq, x_scale, Wq, w_scale, M, N, K, B_pack, R, 0, Y, workspace,
+                       workspace_size, stream);
+}
+
+int sq_lora_delta_from_t(const int8_t *Xq, int64_t M, int64_t N, int64_t K,
+                         const uint16_t *B_pack, int64_t R, float *delta, const void *workspace,
+                         size_t workspace_size, void *stream) {
+  return from_t_common(Xq, nullptr, nullptr, nullptr, M, N, K, B_pack, R, 2, delta, workspace,
                        workspace_size, stream);
 }
 

@@ -34,8 +34,8 @@ static inline int sm_count_of_current_device() {
 }
 
 // LoRA operands of the fused GEMM: T planes [M,R] bf16 (written by the
-// shrink kernel), the packed B [N,R] bf16 and one 16-column-group mask per
-// 128-token tile.
+// shrink kernel), the packed B [N,R] bf16 and one mask of used 16-column
+// groups per 16 tokens.
 struct LoraOperands {
   const uint16_t *T_hi, *T_lo, *B_pack;
   const unsigned long long *mask;
@@ -62,6 +62,12 @@ cudaError_t launch_lora_shrink(const int8_t *Xq, const float *x_scale, int64_t M
                                const int32_t *seg_offsets, const int32_t *seg_adapter, int64_t S,
                                uint16_t *T_hi, uint16_t *T_lo, unsigned long long *mask,
                                cudaStream_t st);
+cudaError_t launch_lora_shrink_raw(const uint16_t *X, int64_t M, int64_t K,
+                                   const uint16_t *A_pack, const int32_t *lora_offset,
+                                   const int32_t *lora_rank, int n_adapters, int64_t R,
+                                   const int32_t *seg_offsets, const int32_t *seg_adapter,
+                                   int64_t S, uint16_t *T_hi, uint16_t *T_lo,
+                                   unsigned long long *mask, cudaStream_t st);
 size_t decode_workspace_bytes(int64_t M);
 bool decode_applicable(int64_t M);
 cudaError_t launch_decode(const int8_t *Xq, const float *x_scale, const int8_t *Wq,

@@ -14,9 +14,14 @@
 // The contraction is a skinny GEMM (N = rank <= 64 per pass) done with
 // warp-level bf16 tensor-core MMAs (m16n8k16, fp32 accumulation): the int8
 // codes are exact in bf16, so converting them in registers loses nothing.
-// Each thread loads 16 contiguous K-bytes of its two rows per 64-wide K chunk;
-// within a chunk the K order seen by the MMA is a permutation that both
-// operands share, which leaves the dot products unchanged.
+// Each thread loads 16 contiguous K values of its two rows per 64-wide K
+// chunk; within a chunk the K order seen by the MMA is a permutation that
+// both operands share, which leaves the dot products unchanged.
+//
+// Raw-input form (the issue's Pitch read on the layer's own activations):
+// T[i, j] = sum_k X[i,k] * A_pack[off_a + j, k] from the bf16 activations,
+// with A_pack holding the adapters as given (packed without the smoothing
+// fold); the bf16 values are the MMA operands directly.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -55,8 +60,8 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
 // c_begin + c_step, ...  acc[nt][.] is the m16n8 fragment of columns
 // [8nt, 8nt+8).  Two chunks are loaded before either is used, so that each
 // warp keeps twice the bytes in flight.
-template <int kNT>
-__device__ __forceinline__ void shrink_warp_tile(const int8_t *__restrict__ Xq, int64_t M,
+template <int kNT, bool kRaw>
+__device__ __forceinline__ void shrink_warp_tile(const void *__restrict__ Xsrc, int64_t M,
                                                  int64_t K, int64_t row0,
                                                  const uint16_t *__restrict__ A_pack, int64_t arow0,
                                                  int c_begin, int c_step, float (&acc)[8][4]) {
@@ -67,18 +72,37 @@ __device__ __forceinline__ void shrink_warp_tile(const int8_t *__restrict__ Xq, 
   for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
     for (int t = 0; t < 4; ++t) acc[nt][t] = 0.f;
-  constexpr int kDepth = (kNT <= 2) ? 4 : ((kNT <= 4) ? 2 : 1);
+  // chunks loaded ahead; the raw form's rows are twice as many bytes
+  constexpr int kDepth0 = (kNT <= 2) ? 4 : ((kNT <= 4) ? 2 : 1);
+  constexpr int kDepth = kRaw ? (kDepth0 > 1 ? kDepth0 / 2 : 1) : kDepth0;
+  constexpr int kXW = kRaw ? 2 : 1;  // 16-byte words per row and chunk
+  const int8_t *Xq = static_cast<const int8_t *>(Xsrc);
+  const uint16_t *Xr = static_cast<const uint16_t *>(Xsrc);
   for (int c0 = c_begin; c0 < nchunks; c0 += kDepth * c_step) {
-    uint4 xa[kDepth], xb[kDepth], bv[kDepth][kNT][2];
+    uint4 xa[kDepth][kXW], xb[kDepth][kXW], bv[kDepth][kNT][2];
 #pragma unroll
     for (int d = 0; d < kDepth; ++d) {
       const int c = c0 + d * c_step;
       const int64_t k = static_cast<int64_t>(c) * 64 + 16 * tig;
       const bool kin = c < nchunks && k < K;  // K % 16 == 0: a 16-slice is all in or out
-      xa[d] = make_uint4(0, 0, 0, 0);
-      xb[d] = make_uint4(0, 0, 0, 0);
-      if (kin && ra < M) xa[d] = __ldg(reinterpret_cast<const uint4 *>(Xq + ra * K + k));
-      if (kin && rb < M) xb[d] = __ldg(reinterpret_cast<const uint4 *>(Xq + rb * K + k));
+#pragma unroll
+      for (int w = 0; w < kXW; ++w) {
+        xa[d][w] = make_uint4(0, 0, 0, 0);
+        xb[d][w] = make_uint4(0, 0, 0, 0);
+      }
+      if constexpr (kRaw) {
+        if (kin && ra < M) {
+          xa[d][0] = __ldg(reinterpret_cast<const uint4 *>(Xr + ra * K + k));
+          xa[d][1] = __ldg(reinterpret_cast<const uint4 *>(Xr + ra * K + k + 8));
+        }
+        if (kin && rb < M) {
+          xb[d][0] = __ldg(reinterpret_cast<const uint4 *>(Xr + rb * K + k));
+          xb[d][1] = __ldg(reinterpret_cast<const uint4 *>(Xr + rb * K + k + 8));
+        }
+      } else {
+        if (kin && ra < M) xa[d][0] = __ldg(reinterpret_cast<const uint4 *>(Xq + ra * K + k));
+        if (kin && rb < M) xb[d][0] = __ldg(reinterpret_cast<const uint4 *>(Xq + rb * K + k));
+      }
 #pragma unroll
       for (int nt = 0; nt < kNT; ++nt) {
         bv[d][nt][0] = make_uint4(0, 0, 0, 0);
@@ -92,15 +116,30 @@ __device__ __forceinline__ void shrink_warp_tile(const int8_t *__restrict__ Xq, 
     }
 #pragma unroll
     for (int d = 0; d < kDepth; ++d) {
-      const uint32_t wa[4] = {xa[d].x, xa[d].y, xa[d].z, xa[d].w};
-      const uint32_t wb[4] = {xb[d].x, xb[d].y, xb[d].z, xb[d].w};
       uint32_t afrag[4][4];  // [k16 step][a0..a3]
+      if constexpr (kRaw) {
+        // elements (4st, 4st+1) and (4st+2, 4st+3) of the 16 are words 2st, 2st+1
+        const uint32_t wa[8] = {xa[d][0].x, xa[d][0].y, xa[d][0].z, xa[d][0].w,
+                                xa[d][1].x, xa[d][1].y, xa[d][1].z, xa[d][1].w};
+        const uint32_t wb[8] = {xb[d][0].x, xb[d][0].y, xb[d][0].z, xb[d][0].w,
+                                xb[d][1].x, xb[d][1].y, xb[d][1].z, xb[d][1].w};
 #pragma unroll
-      for (int st = 0; st < 4; ++st) {
-        afrag[st][0] = bf16x2_of_s8(wa[st], 0);
-        afrag[st][1] = bf16x2_of_s8(wb[st], 0);
-        afrag[st][2] = bf16x2_of_s8(wa[st], 2);
-        afrag[st][3] = bf16x2_of_s8(wb[st], 2);
+        for (int st = 0; st < 4; ++st) {
+          afrag[st][0] = wa[2 * st];
+          afrag[st][1] = wb[2 * st];
+          afrag[st][2] = wa[2 * st + 1];
+          afrag[st][3] = wb[2 * st + 1];
+        }
+      } else {
+        const uint32_t wa[4] = {xa[d][0].x, xa[d][0].y, xa[d][0].z, xa[d][0].w};
+        const uint32_t wb[4] = {xb[d][0].x, xb[d][0].y, xb[d][0].z, xb[d][0].w};
+#pragma unroll
+        for (int st = 0; st < 4; ++st) {
+          afrag[st][0] = bf16x2_of_s8(wa[st], 0);
+          afrag[st][1] = bf16x2_of_s8(wb[st], 0);
+          afrag[st][2] = bf16x2_of_s8(wa[st], 2);
+          afrag[st][3] = bf16x2_of_s8(wb[st], 2);
+        }
       }
 #pragma unroll
       for (int nt = 0; nt < kNT; ++nt) {
@@ -138,9 +177,9 @@ __device__ __forceinline__ void group_sync(int rg, int nwarps) {
     asm volatile("bar.sync %0, %1;" ::"r"(1 + rg), "r"(nwarps * 32) : "memory");
 }
 
-template <int kRG>
+template <int kRG, bool kRaw>
 __global__ void __launch_bounds__(kShrinkThreads) lora_shrink_kernel(
-    const int8_t *__restrict__ Xq, const float *__restrict__ x_scale, int64_t M, int64_t K,
+    const void *__restrict__ Xq, const float *__restrict__ x_scale, int64_t M, int64_t K,
     const uint16_t *__restrict__ A_pack, const int32_t *__restrict__ lora_offset,
     const int32_t *__restrict__ lora_rank, int n_adapters, int64_t R,
     const int32_t *__restrict__ seg_offsets, const int32_t *__restrict__ seg_adapter, int64_t S,
@@ -214,11 +253,11 @@ __global__ void __launch_bounds__(kShrinkThreads) lora_shrink_kernel(
       const int ncols = min(64, rpad - cb);
       float acc[8][4];
       if (ncols <= 16)
-        shrink_warp_tile<2>(Xq, M, K, row0, A_pack, off + cb, ks, kKS, acc);
+        shrink_warp_tile<2, kRaw>(Xq, M, K, row0, A_pack, off + cb, ks, kKS, acc);
       else if (ncols <= 32)
-        shrink_warp_tile<4>(Xq, M, K, row0, A_pack, off + cb, ks, kKS, acc);
+        shrink_warp_tile<4, kRaw>(Xq, M, K, row0, A_pack, off + cb, ks, kKS, acc);
       else
-        shrink_warp_tile<8>(Xq, M, K, row0, A_pack, off + cb, ks, kKS, acc);
+        shrink_warp_tile<8, kRaw>(Xq, M, K, row0, A_pack, off + cb, ks, kKS, acc);
       if (kKS > 1) {
         // fixed-order sum of the group's K parts through shared memory
 #pragma unroll
@@ -255,7 +294,7 @@ __global__ void __launch_bounds__(kShrinkThreads) lora_shrink_kernel(
             const int rr = g + 8 * half;
             const int64_t i = row0 + rr;
             if (!((rows_a >> rr) & 1u) || i >= M) continue;
-            const float xs = x_scale[i];
+            const float xs = kRaw ? 1.0f : x_scale[i];
             const float v0 = (col < rank) ? xs * acc[nt][2 * half] : 0.f;
             const float v1 = (col + 1 < rank) ? xs * acc[nt][2 * half + 1] : 0.f;
             store_t_pair(T_hi, T_lo, i * R + off + col, v0, v1);
@@ -271,13 +310,13 @@ __global__ void __launch_bounds__(kShrinkThreads) lora_shrink_kernel(
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-cudaError_t launch_lora_shrink(const int8_t *Xq, const float *x_scale, int64_t M, int64_t K,
-                               const uint16_t *A_pack, const int32_t *lora_offset,
-                               const int32_t *lora_rank, int n_adapters, int64_t R,
-                               const int32_t *seg_offsets, const int32_t *seg_adapter, int64_t S,
-                               uint16_t *T_hi, uint16_t *T_lo, unsigned long long *mask,
-                               cudaStream_t st) {
-  if (M == 0) return cudaSuccess;
+template <bool kRaw>
+static cudaError_t launch_lora_shrink_t(const void *X, const float *x_scale, int64_t M, int64_t K,
+                                        const uint16_t *A_pack, const int32_t *lora_offset,
+                                        const int32_t *lora_rank, int n_adapters, int64_t R,
+                                        const int32_t *seg_offsets, const int32_t *seg_adapter,
+                                        int64_t S, uint16_t *T_hi, uint16_t *T_lo,
+                                        unsigned long long *mask, cudaStream_t st) {
   const int64_t row_tiles = (M + 15) / 16;
   // widest row grouping that still leaves about two blocks per SM.  Launched
   // in plain stream order: as a programmatic dependent of the quantizer its
@@ -292,26 +331,49 @@ cudaError_t launch_lora_shrink(const int8_t *Xq, const float *x_scale, int64_t M
   cfg.numAttrs = 0;
   if (row_tiles >= 8 * 2 * 148) {
     cfg.gridDim = dim3((g1 + 7) / 8, 1, 1);
-    return cudaLaunchKernelEx(&cfg, lora_shrink_kernel<8>, Xq, x_scale, M, K, A_pack, lora_offset,
-                              lora_rank, n_adapters, R, seg_offsets, seg_adapter, S, T_hi, T_lo,
-                              mask);
+    return cudaLaunchKernelEx(&cfg, lora_shrink_kernel<8, kRaw>, X, x_scale, M, K, A_pack,
+                              lora_offset, lora_rank, n_adapters, R, seg_offsets, seg_adapter, S,
+                              T_hi, T_lo, mask);
   }
   if (row_tiles >= 4 * 2 * 148) {
     cfg.gridDim = dim3((g1 + 3) / 4, 1, 1);
-    return cudaLaunchKernelEx(&cfg, lora_shrink_kernel<4>, Xq, x_scale, M, K, A_pack, lora_offset,
-                              lora_rank, n_adapters, R, seg_offsets, seg_adapter, S, T_hi, T_lo,
-                              mask);
+    return cudaLaunchKernelEx(&cfg, lora_shrink_kernel<4, kRaw>, X, x_scale, M, K, A_pack,
+                              lora_offset, lora_rank, n_adapters, R, seg_offsets, seg_adapter, S,
+                              T_hi, T_lo, mask);
   }
   if (row_tiles >= 2 * 2 * 148) {
     cfg.gridDim = dim3((g1 + 1) / 2, 1, 1);
-    return cudaLaunchKernelEx(&cfg, lora_shrink_kernel<2>, Xq, x_scale, M, K, A_pack, lora_offset,
-                              lora_rank, n_adapters, R, seg_offsets, seg_adapter, S, T_hi, T_lo,
-                              mask);
+    return cudaLaunchKernelEx(&cfg, lora_shrink_kernel<2, kRaw>, X, x_scale, M, K, A_pack,
+                              lora_offset, lora_rank, n_adapters, R, seg_offsets, seg_adapter, S,
+                              T_hi, T_lo, mask);
   }
   cfg.gridDim = dim3(g1, 1, 1);
-  return cudaLaunchKernelEx(&cfg, lora_shrink_kernel<1>, Xq, x_scale, M, K, A_pack, lora_offset,
-                            lora_rank, n_adapters, R, seg_offsets, seg_adapter, S, T_hi, T_lo,
-                            mask);
+  return cudaLaunchKernelEx(&cfg, lora_shrink_kernel<1, kRaw>, X, x_scale, M, K, A_pack,
+                            lora_offset, lora_rank, n_adapters, R, seg_offsets, seg_adapter, S,
+                            T_hi, T_lo, mask);
+}
+
+cudaError_t launch_lora_shrink(const int8_t *Xq, const float *x_scale, int64_t M, int64_t K,
+                               const uint16_t *A_pack, const int32_t *lora_offset,
+                               const int32_t *lora_rank, int n_adapters, int64_t R,
+                               const int32_t *seg_offsets, const int32_t *seg_adapter, int64_t S,
+                               uint16_t *T_hi, uint16_t *T_lo, unsigned long long *mask,
+                               cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  return launch_lora_shrink_t<false>(Xq, x_scale, M, K, A_pack, lora_offset, lora_rank,
+                                     n_adapters, R, seg_offsets, seg_adapter, S, T_hi, T_lo, mask,
+                                     st);
+}
+
+cudaError_t launch_lora_shrink_raw(const uint16_t *X, int64_t M, int64_t K,
+                                   const uint16_t *A_pack, const int32_t *lora_offset,
+                                   const int32_t *lora_rank, int n_adapters, int64_t R,
+                                   const int32_t *seg_offsets, const int32_t *seg_adapter,
+                                   int64_t S, uint16_t *T_hi, uint16_t *T_lo,
+                                   unsigned long long *mask, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  return launch_lora_shrink_t<true>(X, nullptr, M, K, A_pack, lora_offset, lora_rank, n_adapters,
+                                    R, seg_offsets, seg_adapter, S, T_hi, T_lo, mask, st);
 }
 
 }  // namespace sq
