@@ -56,6 +56,8 @@ def lib():
             "sqo_quantize_weight": ([P, P, I64, I64, P, P], None),
             "sqo_quant_act": ([P, I32, P, I64, I64, P, P], None),
             "sqo_prepare_lora": ([P, P, P, I64, I64, I64, F, P, P], None),
+            "sqo_static_act_scale": ([P, P, I64], F),
+            "sqo_quant_act_static": ([P, I32, P, F, I64, I64, P, P], I64),
             "sqo_gemm_rows": ([P, P, I64, I64, I64, P, I64, P], None),
             "sqo_gemm_pairs": ([P, P, I64, P, P, I64, P], None),
             "sqo_token_adapter": ([P, P, I64, I32, I64], I32),
@@ -146,6 +148,25 @@ def quant_act(X: np.ndarray, s: np.ndarray):
     xs = np.zeros(M, np.float32)
     lib().sqo_quant_act(_p(X), _xdtype(X), _p(s), M, K, _p(Xq), _p(xs))
     return Xq, xs
+
+
+def static_act_scale(act_absmax: np.ndarray, s: np.ndarray) -> np.float32:
+    """Per-tensor (static) activation scale from the calibration maxima."""
+    a = _c(act_absmax, np.float32)
+    s = _c(s, np.float32)
+    return np.float32(lib().sqo_static_act_scale(_p(a), _p(s), a.shape[0]))
+
+
+def quant_act_static(X: np.ndarray, s: np.ndarray, scale):
+    """Per-tensor static quantization: (Xq, x_scale [all = scale], clipped count)."""
+    X = np.ascontiguousarray(X)
+    s = _c(s, np.float32)
+    M, K = X.shape
+    Xq = np.zeros((M, K), np.int8)
+    xs = np.zeros(M, np.float32)
+    n = lib().sqo_quant_act_static(_p(X), _xdtype(X), _p(s), float(np.float32(scale)), M, K,
+                                   _p(Xq), _p(xs))
+    return Xq, xs, int(n)
 
 
 def prepare_lora(A: np.ndarray, B: np.ndarray, s: Optional[np.ndarray], lora_alpha: float):

@@ -187,6 +187,45 @@ void sqo_quant_act(const void *X, int dtype, const float *s, int64_t M, int64_t 
   }
 }
 
+/* ---- [SQ] Step 6, per-tensor static level ------------------------------
+ * One activation scale for every token, fixed offline from the calibration
+ * maxima of the smoothed activation ("Calibration in practice": static
+ * scales are the faster, riskier choice):
+ *   scale = RN32( max_j RN32(a_j / s_j) / 127 ).                           */
+float sqo_static_act_scale(const float *act_absmax, const float *s, int64_t K) {
+  double m = 0.0;
+  for (int64_t j = 0; j < K; ++j) {
+    double v = fabs((double)rn32((double)act_absmax[j] / (double)s[j]));
+    if (v > m) m = v;
+  }
+  return rn32(m / 127.0);
+}
+
+/*   xt = RN32(x / s_j);  Xq = clamp(RNE(RN32(xt / scale)), -128, 127);
+ *   x_scale_i = scale for every token.
+ * Returns how many codes the clamp changed (values the calibrated range does
+ * not cover).  scale == 0: every code is 0 and every nonzero xt counts. */
+int64_t sqo_quant_act_static(const void *X, int dtype, const float *s, float scale, int64_t M,
+                             int64_t K, int8_t *Xq, float *x_scale) {
+  int64_t clipped = 0;
+#pragma omp parallel for schedule(static) reduction(+ : clipped)
+  for (int64_t i = 0; i < M; ++i) {
+    x_scale[i] = scale;
+    for (int64_t j = 0; j < K; ++j) {
+      double xt = (double)rn32(x_value(X, dtype, i * K + j) / (double)s[j]);
+      if (scale == 0.0f) {
+        Xq[i * K + j] = 0;
+        if (xt != 0.0) ++clipped;
+        continue;
+      }
+      double r = rne_int((double)rn32(xt / (double)scale));
+      if (r < -128.0 || r > 127.0) ++clipped;
+      Xq[i * K + j] = quant_code(r);
+    }
+  }
+  return clipped;
+}
+
 /* ---- LoRA operands with the smoothing and the scaling folded in ---------
  * The LoRA path consumes the dequantized activations Xq*x_scale, which
  * approximate X/s ([SQ] Step 2); un-smoothing them is folded into A, the same

@@ -30,6 +30,9 @@ void sqo_quantize_weight(const uint16_t *W, const float *s, int64_t N, int64_t K
                          int8_t *Wq, float *w_scale);
 void sqo_quant_act(const void *X, int dtype, const float *s, int64_t M, int64_t K,
                    int8_t *Xq, float *x_scale);
+float sqo_static_act_scale(const float *act_absmax, const float *s, int64_t K);
+int64_t sqo_quant_act_static(const void *X, int dtype, const float *s, float scale, int64_t M,
+                             int64_t K, int8_t *Xq, float *x_scale);
 void sqo_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s, int64_t r,
                       int64_t K, int64_t N, float lora_alpha, uint16_t *A_s,
                       uint16_t *B_s);
