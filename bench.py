@@ -53,6 +53,9 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wk.SPECS))
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--act-quant", choices=["dynamic", "static"], default="dynamic",
+                   help="per-token scales (default) or one calibrated per-tensor scale "
+                        "(sq_quant_act_static)")
     p.add_argument("--lora-input", choices=["dequant", "raw"], default="dequant",
                    help="what the LoRA path reads: the dequantized codes (default) or the "
                         "raw bf16 activations (sq_lora_shrink_raw + sq_linear_lora_from_t)")
@@ -326,8 +329,17 @@ def run_ours(args):
         flush.fill_(v)
         flush_read.max()
 
+    static = args.act_quant == "static"
+    if static:
+        static_scale = torch.empty(1, dtype=torch.float32, device=dev)
+        sq.sq_static_act_scale(act_absmax, s, static_scale)
+        clip_count = torch.zeros(1, dtype=torch.int64, device=dev)
+
     def step():
-        sq.sq_quant_act(X, s, Xq, x_scale)
+        if static:
+            sq.sq_quant_act_static(X, s, static_scale, Xq, x_scale, clip_count)
+        else:
+            sq.sq_quant_act(X, s, Xq, x_scale)
         if raw:
             sq.sq_lora_shrink_raw(X, lora, seg_offsets, seg_adapter, ws)
             sq.sq_linear_lora_from_t(Xq, x_scale, Wq, w_scale, lora, Y, ws)
@@ -440,9 +452,11 @@ def run_ours(args):
         "config": {"workload": wl.spec.name, "M": M, "K": K, "N": N,
                    "adapters": len(wl.adapters), "ranks": sorted(set(a.r for a in wl.adapters)),
                    "segments": int(len(wl.seg_adapter)), "alpha": wl.alpha,
-                   "step": ("sq_quant_act + sq_lora_shrink_raw + sq_linear_lora_from_t "
-                            "(LoRA on the raw bf16 activations)" if raw else
-                            "sq_quant_act + sq_linear_lora (shrink + fused GEMM)"),
+                   "step": (("sq_quant_act_static" if static else "sq_quant_act") +
+                            (" + sq_lora_shrink_raw + sq_linear_lora_from_t "
+                             "(LoRA on the raw bf16 activations)" if raw else
+                             " + sq_linear_lora (shrink + fused GEMM)")),
+                   "act_quant": args.act_quant,
                    "l2": "flushed between timed steps (256 MiB write + 256 MiB read, untimed)",
                    "parallelism": f"replicas x{world}"},
         "tokens_per_s": tok_s,

@@ -161,6 +161,25 @@ int sq_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s, int64_
 int sq_quant_act(const void *X, int x_dtype, const float *s, int64_t M, int64_t K,
                  int8_t *Xq, float *x_scale, void *stream);
 
+/* Per-tensor static level of Step 6 ("SmoothQuant" explainer, Step 6 and
+ * "Calibration in practice": one activation scale for every token, fixed
+ * offline from the calibration range; faster, and values outside the
+ * calibrated range are clipped).
+ * sq_static_act_scale: *scale = RN(max_j RN(act_absmax_j / s_j) / 127), IEEE
+ * fp32 divisions.  act_absmax, s: [K] f32 device; scale: one f32, device. */
+int sq_static_act_scale(const float *act_absmax, const float *s, int64_t K, float *scale,
+                        void *stream);
+
+/* xt = RN(X[i,j] / s_j);  Xq = clamp(round_half_even(RN(xt / scale)), -128, 127);
+ * x_scale[i] = scale for every token (so sq_linear_lora takes it unchanged);
+ * *clip_count += the number of codes the clamp changed (scale == 0: codes 0,
+ * every nonzero xt counts).  scale: one f32 (device, e.g. from
+ * sq_static_act_scale); clip_count: one u64 (device, 8-byte aligned; zero it
+ * before a run to count that run).  Bit-exact. */
+int sq_quant_act_static(const void *X, int x_dtype, const float *s, const float *scale,
+                        int64_t M, int64_t K, int8_t *Xq, float *x_scale,
+                        unsigned long long *clip_count, void *stream);
+
 /* Bytes of device workspace sq_linear_lora needs for M tokens and a LoRA
  * pack of width R (0 when R == 0). */
 size_t sq_linear_lora_workspace_size(int64_t M, int64_t R);

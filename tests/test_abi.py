@@ -143,3 +143,17 @@ def test_raw_lora_entry_validation(lib):
     assert h(A, 64, 128, 1024, A, 32, A, A, tws, None) in (CUDA, DEVICE)
     # s == NULL is the raw-input packing (A unchanged), not an argument error
     assert lib.sq_prepare_lora(A, A, None, 8, 64, 32, 16.0, 16, 0, A, A, None) in (CUDA, DEVICE)
+
+
+def test_static_quant_entry_validation(lib):
+    assert lib.sq_static_act_scale(A, A, 1000, A, None) == SHAPE        # K % 16
+    assert lib.sq_static_act_scale(A, A, 0, A, None) == INVALID
+    assert lib.sq_static_act_scale(A, A, 64, A + 2, None) == INVALID    # scale alignment
+    assert lib.sq_static_act_scale(A, A, 64, A, None) in (CUDA, DEVICE)
+    f = lib.sq_quant_act_static
+    assert f(A, 1, A, A, 64, 1000, A, A, A, None) == SHAPE               # K % 16
+    assert f(A, 7, A, A, 64, 1024, A, A, A, None) == INVALID             # dtype
+    assert f(A, 1, A, A, 64, 1024, A, A, A + 4, None) == INVALID         # counter alignment
+    assert f(A, 1, A, None, 64, 1024, A, A, A, None) == INVALID
+    assert f(A + 2, 1, A, A, 64, 1024, A, A, A, None) == INVALID
+    assert f(A, 1, A, A, 64, 1024, A, A, A, None) in (CUDA, DEVICE)

@@ -23,7 +23,7 @@ __all__ = [
     "sq_compute_smoothing", "sq_quantize_weight", "sq_prepare_lora", "sq_quant_act",
     "sq_linear_lora_workspace_size", "sq_linear_lora", "sq_linear_lora_noalloc", "sq_gemm_i32",
     "sq_lora_delta", "sq_lora_t_workspace_size", "sq_lora_shrink_raw", "sq_linear_lora_from_t",
-    "sq_lora_delta_from_t",
+    "sq_lora_delta_from_t", "sq_static_act_scale", "sq_quant_act_static",
 ]
 
 SQ_DTYPE_F32 = 0
@@ -134,6 +134,20 @@ def sq_prepare_lora(A, B, s, lora_alpha: float, R: int, off: int, A_pack, B_pack
     N = B.shape[0]
     _check(_lib().sq_prepare_lora(_ptr(A), _ptr(B), _ptr(s), r, K, N, float(lora_alpha), R, off,
                                   _ptr(A_pack), _ptr(B_pack), _stream(stream)), "sq_prepare_lora")
+
+
+def sq_static_act_scale(act_absmax, s, scale, stream=None) -> None:
+    """Per-tensor static activation scale (one f32 device tensor) from calibration maxima."""
+    _check(_lib().sq_static_act_scale(_ptr(act_absmax), _ptr(s), act_absmax.shape[0], _ptr(scale),
+                                      _stream(stream)), "sq_static_act_scale")
+
+
+def sq_quant_act_static(X, s, scale, Xq, x_scale, clip_count, stream=None) -> None:
+    """Per-tensor static quantization; clip_count (one int64 device tensor) is incremented."""
+    M, K = X.shape
+    _check(_lib().sq_quant_act_static(_ptr(X), _xdtype(X), _ptr(s), _ptr(scale), M, K, _ptr(Xq),
+                                      _ptr(x_scale), _ptr(clip_count), _stream(stream)),
+           "sq_quant_act_static")
 
 
 def sq_quant_act(X, s, Xq, x_scale, stream=None) -> None:

@@ -247,6 +247,36 @@ int sq_quant_act(const void *X, int x_dtype, const float *s, int64_t M, int64_t 
       launch_quant_act(X, x_dtype, s, M, K, Xq, x_scale, static_cast<cudaStream_t>(stream)));
 }
 
+static bool aligned_to(const void *p, uintptr_t a) {
+  return p != nullptr && (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+int sq_static_act_scale(const float *act_absmax, const float *s, int64_t K, float *scale,
+                        void *stream) {
+  int st = check_mk(1, K);
+  if (st) return st;
+  if (K == 0 || !ptr_ok(act_absmax) || !ptr_ok(s) || !aligned_to(scale, 4))
+    return SQ_ERR_INVALID_ARG;
+  if ((st = check_device())) return st;
+  return cuda_status(
+      launch_static_act_scale(act_absmax, s, K, scale, static_cast<cudaStream_t>(stream)));
+}
+
+int sq_quant_act_static(const void *X, int x_dtype, const float *s, const float *scale,
+                        int64_t M, int64_t K, int8_t *Xq, float *x_scale,
+                        unsigned long long *clip_count, void *stream) {
+  int st = check_mk(M, K);
+  if (st) return st;
+  if (x_dtype != SQ_DTYPE_BF16 && x_dtype != SQ_DTYPE_F32) return SQ_ERR_INVALID_ARG;
+  if (!aligned_to(scale, 4) || !aligned_to(clip_count, 8)) return SQ_ERR_INVALID_ARG;
+  if (M > 0 && (!ptr_ok(x_scale) || (K > 0 && (!ptr_ok(X) || !ptr_ok(s) || !ptr_ok(Xq)))))
+    return SQ_ERR_INVALID_ARG;
+  if ((st = check_device())) return st;
+  // (K == 0: no codes, the scale is still every token's scale)
+  return cuda_status(launch_quant_act_static(X, x_dtype, s, scale, M, K, Xq, x_scale, clip_count,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
 size_t sq_linear_lora_workspace_size(int64_t M, int64_t R) { return workspace_bytes(M, R); }
 
 static int linear_common(const int8_t *Xq, const float *x_scale, const int8_t *Wq,

@@ -51,6 +51,11 @@ cudaError_t launch_compute_smoothing(const float *a, const float *w, int64_t K, 
                                      float *s, cudaStream_t st);
 cudaError_t launch_quant_act(const void *X, int dtype, const float *s, int64_t M, int64_t K,
                              int8_t *Xq, float *x_scale, cudaStream_t st);
+cudaError_t launch_static_act_scale(const float *a, const float *s, int64_t K, float *scale,
+                                    cudaStream_t st);
+cudaError_t launch_quant_act_static(const void *X, int dtype, const float *s, const float *scale,
+                                    int64_t M, int64_t K, int8_t *Xq, float *x_scale,
+                                    unsigned long long *clip_count, cudaStream_t st);
 cudaError_t launch_quantize_weight(const uint16_t *W, const float *s, int64_t N, int64_t K,
                                    int8_t *Wq, float *w_scale, cudaStream_t st);
 cudaError_t launch_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s, int64_t r,
