@@ -321,6 +321,27 @@ def smoothed_product_rows(X, W, s, rows: Optional[Sequence[int]] = None) -> np.n
     return Y
 
 
+def alpha_output_error(X, W, alpha: float, rows: Optional[Sequence[int]] = None):
+    """Layer-wise output error of the W8A8 layer for one alpha, on the
+    calibration tokens X themselves ("Reading the diagnostics": compare
+    layer-wise output error across alpha values; "Per-layer alpha").
+
+    a = per-channel max |X|, w = per-channel max |W|, s = smoothing(a, w, alpha),
+    Y = dequantized W8A8 output (fp64), Y_ref = X W^T (fp64).
+    Returns (sum over rows of (Y - Y_ref)^2, sum of Y_ref^2)."""
+    X = np.ascontiguousarray(X)
+    a = act_absmax_update(X)
+    s = compute_smoothing(a, weight_absmax(W), alpha)
+    Wq, ws = quantize_weight(W, s)
+    Xq, xs = quant_act(X, s)
+    M = X.shape[0]
+    rows = np.arange(M, dtype=np.int64) if rows is None else _c(rows, np.int64)
+    none = np.array([0, M], np.int32), np.array([-1], np.int32)
+    Y = linear_lora_rows(Xq, xs, Wq, ws, [], [], none[0], none[1], rows, want=("Y",))["Y"]
+    ref = reference_rows(X, W, [], [], [], none[0], none[1], rows)
+    return float(((Y - ref) ** 2).sum()), float((ref ** 2).sum())
+
+
 class Prepared:
     """Everything the oracle derives offline and on the hot path for one workload."""
 
