@@ -247,6 +247,25 @@ int sq_lora_delta(const int8_t *Xq, const float *x_scale, int64_t M, int64_t N,
                   void *stream);
 
 /* ---------------------------------------------------------------------------
+ * Offline diagnostic: layer-wise output error for one migration strength
+ * ("SmoothQuant" explainer, "Reading the diagnostics": compare layer-wise
+ * output error across alpha values; "Variants and related ideas": choose
+ * alpha layer by layer by calibration error).  On the calibration tokens X
+ * [M,K] (bf16 or f32, device) and the weights W [N,K] bf16 (device): the
+ * calibration maxima of X and W, s(alpha), the quantized weights and
+ * activations and the fused GEMM's Y (bf16, no adapters), then
+ *   err[0] = sum (Y - X W^T)^2,  err[1] = sum (X W^T)^2
+ * with X W^T from the unquantized operands (fp32 products and sums, fp64
+ * totals).  err: two doubles, device, overwritten.  alpha in [0, 1].
+ * workspace: >= sq_alpha_error_workspace_size(M, N, K) bytes, 256-byte
+ * aligned device memory (scratch).  Errors: SQ_ERR_INVALID_ARG,
+ * SQ_ERR_UNSUPPORTED_SHAPE (K % 16, N % 16), SQ_ERR_WORKSPACE. */
+size_t sq_alpha_error_workspace_size(int64_t M, int64_t N, int64_t K);
+int sq_alpha_output_error(const void *X, int x_dtype, const uint16_t *W, int64_t M, int64_t N,
+                          int64_t K, float alpha, double *err, void *workspace,
+                          size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------
  * Raw-input reading of the LoRA path ("[Feature]: LoRA support for W8A8
  * SmoothQuant", Pitch: the low-rank path runs in BF16 after the INT8 GEMM
  * and is added to the dequantized output), taken on the layer's own bf16

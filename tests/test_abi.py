@@ -157,3 +157,16 @@ def test_static_quant_entry_validation(lib):
     assert f(A, 1, A, None, 64, 1024, A, A, A, None) == INVALID
     assert f(A + 2, 1, A, A, 64, 1024, A, A, A, None) == INVALID
     assert f(A, 1, A, A, 64, 1024, A, A, A, None) in (CUDA, DEVICE)
+
+
+def test_alpha_error_entry_validation(lib):
+    assert lib.sq_alpha_error_workspace_size(0, 64, 64) == 0
+    wsz = lib.sq_alpha_error_workspace_size(64, 128, 256)
+    assert wsz >= 128 * 256 + 64 * 256 + 2 * 64 * 128 and wsz % 256 == 0
+    f = lib.sq_alpha_output_error
+    assert f(A, 1, A, 64, 128, 1000, 0.5, A, A, wsz, None) == SHAPE    # K % 16
+    assert f(A, 1, A, 64, 100, 256, 0.5, A, A, wsz, None) == SHAPE     # N % 16
+    assert f(A, 1, A, 64, 128, 256, 1.5, A, A, wsz, None) == INVALID   # alpha
+    assert f(A, 1, A, 64, 128, 256, 0.5, A + 4, A, wsz, None) == INVALID  # err alignment
+    assert f(A, 1, A, 64, 128, 256, 0.5, A, A, wsz - 1, None) == WORKSPACE
+    assert f(A, 1, A, 64, 128, 256, 0.5, A, A, wsz, None) in (CUDA, DEVICE)

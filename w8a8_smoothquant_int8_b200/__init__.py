@@ -24,6 +24,7 @@ __all__ = [
     "sq_linear_lora_workspace_size", "sq_linear_lora", "sq_linear_lora_noalloc", "sq_gemm_i32",
     "sq_lora_delta", "sq_lora_t_workspace_size", "sq_lora_shrink_raw", "sq_linear_lora_from_t",
     "sq_lora_delta_from_t", "sq_static_act_scale", "sq_quant_act_static",
+    "sq_alpha_error_workspace_size", "sq_alpha_output_error", "alpha_sweep",
 ]
 
 SQ_DTYPE_F32 = 0
@@ -243,6 +244,38 @@ def sq_gemm_i32(Xq, Wq, acc, stream=None) -> None:
     M, K = Xq.shape
     N = Wq.shape[0]
     _check(_lib().sq_gemm_i32(_ptr(Xq), _ptr(Wq), M, N, K, _ptr(acc), _stream(stream)), "sq_gemm_i32")
+
+
+def sq_alpha_error_workspace_size(M: int, N: int, K: int) -> int:
+    return int(_lib().sq_alpha_error_workspace_size(M, N, K))
+
+
+def sq_alpha_output_error(X, W, alpha: float, err, workspace, stream=None) -> None:
+    """err (2 float64, device) = (sum (Y - X W^T)^2, sum (X W^T)^2) for one alpha."""
+    M, K = X.shape
+    N = W.shape[0]
+    wp, wb = _ws(workspace)
+    _check(_lib().sq_alpha_output_error(_ptr(X), _xdtype(X), _ptr(W), M, N, K, float(alpha),
+                                        _ptr(err), wp, wb, _stream(stream)),
+           "sq_alpha_output_error")
+
+
+def alpha_sweep(X_cal, W, alphas: Sequence[float], stream=None):
+    """Per-layer migration strength by calibration error: the relative
+    squared output error ||Y - X W^T||^2 / ||X W^T||^2 of the W8A8 layer for
+    each alpha, on the calibration tokens.  Returns (errors, best alpha)."""
+    import torch
+    M, K = X_cal.shape
+    N = W.shape[0]
+    ws = torch.empty(max(sq_alpha_error_workspace_size(M, N, K), 256), dtype=torch.uint8,
+                     device=X_cal.device)
+    err = torch.empty((len(alphas), 2), dtype=torch.float64, device=X_cal.device)
+    for i, a in enumerate(alphas):
+        sq_alpha_output_error(X_cal, W, a, err[i], ws, stream)
+    e = err.cpu()
+    rel = [float(e[i, 0] / e[i, 1]) if float(e[i, 1]) > 0 else 0.0 for i in range(len(alphas))]
+    best = min(range(len(alphas)), key=lambda i: rel[i]) if alphas else -1
+    return rel, (float(alphas[best]) if best >= 0 else None)
 
 
 def sq_lora_t_workspace_size(M: int, R: int) -> int:

@@ -364,6 +364,28 @@ int sq_lora_delta(const int8_t *Xq, const float *x_scale, int64_t M, int64_t N, 
                        workspace_size, stream);
 }
 
+// ---- layer-wise output error for one alpha (offline diagnostic) ------------
+size_t sq_alpha_error_workspace_size(int64_t M, int64_t N, int64_t K) {
+  return alpha_error_workspace_bytes(M, N, K);
+}
+
+int sq_alpha_output_error(const void *X, int x_dtype, const uint16_t *W, int64_t M, int64_t N,
+                          int64_t K, float alpha, double *err, void *workspace,
+                          size_t workspace_size, void *stream) {
+  int st = check_mk(M, K);
+  if (st) return st;
+  if (x_dtype != SQ_DTYPE_BF16 && x_dtype != SQ_DTYPE_F32) return SQ_ERR_INVALID_ARG;
+  if (!(alpha >= 0.0f && alpha <= 1.0f) || M <= 0 || N <= 0 || K <= 0) return SQ_ERR_INVALID_ARG;
+  if (N % 16 != 0) return SQ_ERR_UNSUPPORTED_SHAPE;
+  if (!ptr_ok(X) || !ptr_ok(W) || !aligned_to(err, 8)) return SQ_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_size < alpha_error_workspace_bytes(M, N, K))
+    return SQ_ERR_WORKSPACE;
+  if ((st = check_device())) return st;
+  return cuda_status(launch_alpha_error(X, x_dtype, W, M, N, K, alpha, err, workspace,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 // ---- raw-input reading of the LoRA path ------------------------------------
 size_t sq_lora_t_workspace_size(int64_t M, int64_t R) { return t_workspace_bytes(M, R); }
 

@@ -85,6 +85,11 @@ cudaError_t launch_w8a8_gemm(const int8_t *Xq, const int8_t *Wq, const float *x_
                              const float *w_scale, int64_t M, int64_t N, int64_t K, int mode,
                              void *out, const LoraOperands *lora, cudaStream_t st);
 
+size_t alpha_error_workspace_bytes(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_alpha_error(const void *X, int dtype, const uint16_t *W, int64_t M, int64_t N,
+                               int64_t K, float alpha, double *err, void *workspace,
+                               cudaStream_t st);
+
 // Adapter of token `i` for a segment table: the first segment s with
 // off[s] <= i < off[s+1].  Segments are assumed sorted (off non-decreasing);
 // the binary search finds the last segment starting at or before i and then

@@ -4,5 +4,6 @@
 #include "lora_shrink.cu"
 #include "gemm_sm100.cu"
 #include "decode.cu"
+#include "alpha_error.cu"
 #include "api.cu"
 #include "noalloc.cu"
