@@ -57,6 +57,8 @@ def lib():
             "sqo_quant_act": ([P, I32, P, I64, I64, P, P], None),
             "sqo_prepare_lora": ([P, P, P, I64, I64, I64, F, P, P], None),
             "sqo_static_act_scale": ([P, P, I64], F),
+            "sqo_fold_norm_weight": ([P, P, I64, P], None),
+            "sqo_rmsnorm_quant_act": ([P, P, F, I64, I64, P, P], None),
             "sqo_quant_act_static": ([P, I32, P, F, I64, I64, P, P], I64),
             "sqo_gemm_rows": ([P, P, I64, I64, I64, P, I64, P], None),
             "sqo_gemm_pairs": ([P, P, I64, P, P, I64, P], None),
@@ -167,6 +169,26 @@ def quant_act_static(X: np.ndarray, s: np.ndarray, scale):
     n = lib().sqo_quant_act_static(_p(X), _xdtype(X), _p(s), float(np.float32(scale)), M, K,
                                    _p(Xq), _p(xs))
     return Xq, xs, int(n)
+
+
+def fold_norm_weight(gamma: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """gamma_s = RN32(gamma / s): Step 5's inverse scale folded into a norm weight."""
+    g = _c(gamma, np.float32)
+    s = _c(s, np.float32)
+    out = np.zeros_like(g)
+    lib().sqo_fold_norm_weight(_p(g), _p(s), g.shape[0], _p(out))
+    return out
+
+
+def rmsnorm_quant_act(H: np.ndarray, gamma_s: np.ndarray, eps: float):
+    """RMS normalization with the folded weight, then per-token INT8 (bf16 H)."""
+    H = _c(H, np.uint16)
+    g = _c(gamma_s, np.float32)
+    M, K = H.shape
+    Xq = np.zeros((M, K), np.int8)
+    xs = np.zeros(M, np.float32)
+    lib().sqo_rmsnorm_quant_act(_p(H), _p(g), float(np.float32(eps)), M, K, _p(Xq), _p(xs))
+    return Xq, xs
 
 
 def prepare_lora(A: np.ndarray, B: np.ndarray, s: Optional[np.ndarray], lora_alpha: float):

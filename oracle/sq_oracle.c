@@ -226,6 +226,43 @@ int64_t sqo_quant_act_static(const void *X, int dtype, const float *s, float sca
   return clipped;
 }
 
+/* ---- [SQ] Step 5: the inverse scale folded into the normalization weight -
+ * "The inverse scale can be folded into the normalization layer's weights":
+ *   gamma_s[j] = RN32(gamma[j] / s_j)                                       */
+void sqo_fold_norm_weight(const float *gamma, const float *s, int64_t K, float *gamma_s) {
+  for (int64_t j = 0; j < K; ++j) gamma_s[j] = rn32((double)gamma[j] / (double)s[j]);
+}
+
+/* RMS normalization with the folded weight, then Step 6 per token:
+ *   r_i  = RN32( 1 / sqrt( (sum_j h_ij^2) / K + eps ) )   (fp64 inside)
+ *   xt   = RN32( RN32(h_ij * r_i) * gamma_s[j] )
+ *   x_scale_i = RN32(max_j |xt| / 127),  Xq = clamp(RNE(RN32(xt / x_scale_i)))
+ * H [M,K] bf16.  The sum of squares of bf16 values is exact in fp64 whenever
+ * a row's squares span less than 2^37 in magnitude; it is summed in order. */
+void sqo_rmsnorm_quant_act(const uint16_t *H, const float *gamma_s, float eps, int64_t M,
+                           int64_t K, int8_t *Xq, float *x_scale) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < M; ++i) {
+    double ss = 0.0;
+    for (int64_t j = 0; j < K; ++j) {
+      double h = bf16_value(H[i * K + j]);
+      ss += h * h;
+    }
+    float r = rn32(1.0 / sqrt(ss / (double)K + (double)eps));
+    double amax = 0.0;
+    for (int64_t j = 0; j < K; ++j) {
+      double xt = (double)rn32((double)rn32(bf16_value(H[i * K + j]) * (double)r) * (double)gamma_s[j]);
+      if (fabs(xt) > amax) amax = fabs(xt);
+    }
+    float sc = rn32(amax / 127.0);
+    x_scale[i] = sc;
+    for (int64_t j = 0; j < K; ++j) {
+      double xt = (double)rn32((double)rn32(bf16_value(H[i * K + j]) * (double)r) * (double)gamma_s[j]);
+      Xq[i * K + j] = (sc == 0.0f) ? 0 : quant_code((double)rn32(xt / (double)sc));
+    }
+  }
+}
+
 /* ---- LoRA operands with the smoothing and the scaling folded in ---------
  * The LoRA path consumes the dequantized activations Xq*x_scale, which
  * approximate X/s ([SQ] Step 2); un-smoothing them is folded into A, the same

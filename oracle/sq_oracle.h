@@ -33,6 +33,9 @@ void sqo_quant_act(const void *X, int dtype, const float *s, int64_t M, int64_t 
 float sqo_static_act_scale(const float *act_absmax, const float *s, int64_t K);
 int64_t sqo_quant_act_static(const void *X, int dtype, const float *s, float scale, int64_t M,
                              int64_t K, int8_t *Xq, float *x_scale);
+void sqo_fold_norm_weight(const float *gamma, const float *s, int64_t K, float *gamma_s);
+void sqo_rmsnorm_quant_act(const uint16_t *H, const float *gamma_s, float eps, int64_t M,
+                           int64_t K, int8_t *Xq, float *x_scale);
 void sqo_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s, int64_t r,
                       int64_t K, int64_t N, float lora_alpha, uint16_t *A_s,
                       uint16_t *B_s);
