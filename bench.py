@@ -56,6 +56,10 @@ def parse():
     p.add_argument("--act-quant", choices=["dynamic", "static"], default="dynamic",
                    help="per-token scales (default) or one calibrated per-tensor scale "
                         "(sq_quant_act_static)")
+    p.add_argument("--norm-fold", action="store_true",
+                   help="the activations are a normalization's input: RMS norm with 1/s folded "
+                        "into its weight, fused with the per-token quantization "
+                        "(sq_rmsnorm_quant_act)")
     p.add_argument("--lora-input", choices=["dequant", "raw"], default="dequant",
                    help="what the LoRA path reads: the dequantized codes (default) or the "
                         "raw bf16 activations (sq_lora_shrink_raw + sq_linear_lora_from_t)")
@@ -330,13 +334,21 @@ def run_ours(args):
         flush_read.max()
 
     static = args.act_quant == "static"
+    norm = args.norm_fold
+    if norm:
+        if static or not wl.x_is_bf16:
+            raise SystemExit("--norm-fold takes bf16 activations and per-token scales")
+        gamma_s = torch.empty(K, dtype=torch.float32, device=dev)
+        sq.sq_fold_norm_weight(torch.from_numpy(wk.norm_gamma(K, wl.seed)).to(dev), s, gamma_s)
     if static:
         static_scale = torch.empty(1, dtype=torch.float32, device=dev)
         sq.sq_static_act_scale(act_absmax, s, static_scale)
         clip_count = torch.zeros(1, dtype=torch.int64, device=dev)
 
     def step():
-        if static:
+        if norm:
+            sq.sq_rmsnorm_quant_act(X, gamma_s, 1e-6, Xq, x_scale)
+        elif static:
             sq.sq_quant_act_static(X, s, static_scale, Xq, x_scale, clip_count)
         else:
             sq.sq_quant_act(X, s, Xq, x_scale)
@@ -452,7 +464,8 @@ def run_ours(args):
         "config": {"workload": wl.spec.name, "M": M, "K": K, "N": N,
                    "adapters": len(wl.adapters), "ranks": sorted(set(a.r for a in wl.adapters)),
                    "segments": int(len(wl.seg_adapter)), "alpha": wl.alpha,
-                   "step": (("sq_quant_act_static" if static else "sq_quant_act") +
+                   "step": (("sq_rmsnorm_quant_act" if norm else
+                             "sq_quant_act_static" if static else "sq_quant_act") +
                             (" + sq_lora_shrink_raw + sq_linear_lora_from_t "
                              "(LoRA on the raw bf16 activations)" if raw else
                              " + sq_linear_lora (shrink + fused GEMM)")),

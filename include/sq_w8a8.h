@@ -180,6 +180,25 @@ int sq_quant_act_static(const void *X, int x_dtype, const float *s, const float 
                         int64_t M, int64_t K, int8_t *Xq, float *x_scale,
                         unsigned long long *clip_count, void *stream);
 
+/* Step 5 with a normalization in front of the layer ("the inverse scale can
+ * be folded into the normalization layer's weights"):
+ * sq_fold_norm_weight: gamma_s[j] = RN(gamma[j] / s_j) (IEEE fp32 division;
+ * offline).  gamma, s, gamma_s: [K] f32 device. */
+int sq_fold_norm_weight(const float *gamma, const float *s, int64_t K, float *gamma_s,
+                        void *stream);
+
+/* RMS normalization with the folded weight fused with Step 6 (per token):
+ *   r_i = RN32(1 / sqrt(sum_j H[i,j]^2 / K + eps))  (fp64 sum of the exact
+ *         squares, correctly rounded sqrt and division),
+ *   xt = RN(RN(H[i,j] * r_i) * gamma_s[j]);  x_scale_i = RN(max_j |xt| / 127);
+ *   Xq = clamp(round_half_even(RN(xt / x_scale_i)), -128, 127).
+ * H [M,K] bf16 (the layer's pre-normalization input), device.  Bit-exact
+ * while a row's squares span less than 2^37 (the fp64 sum is then exact, so
+ * its order does not matter).  K % 16 == 0 and K <= 32768, else
+ * SQ_ERR_UNSUPPORTED_SHAPE; eps >= 0. */
+int sq_rmsnorm_quant_act(const uint16_t *H, const float *gamma_s, float eps, int64_t M, int64_t K,
+                         int8_t *Xq, float *x_scale, void *stream);
+
 /* Bytes of device workspace sq_linear_lora needs for M tokens and a LoRA
  * pack of width R (0 when R == 0). */
 size_t sq_linear_lora_workspace_size(int64_t M, int64_t R);

@@ -170,3 +170,15 @@ def test_alpha_error_entry_validation(lib):
     assert f(A, 1, A, 64, 128, 256, 0.5, A + 4, A, wsz, None) == INVALID  # err alignment
     assert f(A, 1, A, 64, 128, 256, 0.5, A, A, wsz - 1, None) == WORKSPACE
     assert f(A, 1, A, 64, 128, 256, 0.5, A, A, wsz, None) in (CUDA, DEVICE)
+
+
+def test_norm_fold_entry_validation(lib):
+    assert lib.sq_fold_norm_weight(A, A, 1000, A, None) == SHAPE
+    assert lib.sq_fold_norm_weight(A + 4, A, 64, A, None) == INVALID
+    assert lib.sq_fold_norm_weight(A, A, 64, A, None) in (CUDA, DEVICE)
+    f = lib.sq_rmsnorm_quant_act
+    assert f(A, A, 1e-6, 64, 1000, A, A, None) == SHAPE         # K % 16
+    assert f(A, A, 1e-6, 64, 65536, A, A, None) == SHAPE        # beyond 32768 channels
+    assert f(A, A, -1.0, 64, 1024, A, A, None) == INVALID       # eps < 0
+    assert f(A + 2, A, 1e-6, 64, 1024, A, A, None) == INVALID
+    assert f(A, A, 1e-6, 64, 1024, A, A, None) in (CUDA, DEVICE)

@@ -25,6 +25,7 @@ __all__ = [
     "sq_lora_delta", "sq_lora_t_workspace_size", "sq_lora_shrink_raw", "sq_linear_lora_from_t",
     "sq_lora_delta_from_t", "sq_static_act_scale", "sq_quant_act_static",
     "sq_alpha_error_workspace_size", "sq_alpha_output_error", "alpha_sweep",
+    "sq_fold_norm_weight", "sq_rmsnorm_quant_act",
 ]
 
 SQ_DTYPE_F32 = 0
@@ -149,6 +150,19 @@ def sq_quant_act_static(X, s, scale, Xq, x_scale, clip_count, stream=None) -> No
     _check(_lib().sq_quant_act_static(_ptr(X), _xdtype(X), _ptr(s), _ptr(scale), M, K, _ptr(Xq),
                                       _ptr(x_scale), _ptr(clip_count), _stream(stream)),
            "sq_quant_act_static")
+
+
+def sq_fold_norm_weight(gamma, s, gamma_s, stream=None) -> None:
+    """gamma_s = gamma / s (the smoothing folded into an RMS-norm weight)."""
+    _check(_lib().sq_fold_norm_weight(_ptr(gamma), _ptr(s), gamma.shape[0], _ptr(gamma_s),
+                                      _stream(stream)), "sq_fold_norm_weight")
+
+
+def sq_rmsnorm_quant_act(H, gamma_s, eps: float, Xq, x_scale, stream=None) -> None:
+    """RMS normalization with the folded weight fused with per-token INT8."""
+    M, K = H.shape
+    _check(_lib().sq_rmsnorm_quant_act(_ptr(H), _ptr(gamma_s), float(eps), M, K, _ptr(Xq),
+                                       _ptr(x_scale), _stream(stream)), "sq_rmsnorm_quant_act")
 
 
 def sq_quant_act(X, s, Xq, x_scale, stream=None) -> None:

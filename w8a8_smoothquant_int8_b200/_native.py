@@ -41,6 +41,8 @@ SIGNATURES = {
     "sq_gemm_i32": ([P, P, I64, I64, I64, P, P], I32),
     "sq_lora_delta": ([P, P, I64, I64, I64, P, P, P, P, I32, I64, P, P, I64, P, P, SZ, P], I32),
     "sq_lora_t_workspace_size": ([I64, I64], SZ),
+    "sq_fold_norm_weight": ([P, P, I64, P, P], I32),
+    "sq_rmsnorm_quant_act": ([P, P, F32, I64, I64, P, P, P], I32),
     "sq_alpha_error_workspace_size": ([I64, I64, I64], SZ),
     "sq_alpha_output_error": ([P, I32, P, I64, I64, I64, F32, P, P, SZ, P], I32),
     "sq_static_act_scale": ([P, P, I64, P, P], I32),

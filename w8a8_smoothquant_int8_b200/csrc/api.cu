@@ -277,6 +277,30 @@ int sq_quant_act_static(const void *X, int x_dtype, const float *s, const float 
                                              static_cast<cudaStream_t>(stream)));
 }
 
+int sq_fold_norm_weight(const float *gamma, const float *s, int64_t K, float *gamma_s,
+                        void *stream) {
+  int st = check_mk(1, K);
+  if (st) return st;
+  if (K > 0 && (!ptr_ok(gamma) || !ptr_ok(s) || !ptr_ok(gamma_s))) return SQ_ERR_INVALID_ARG;
+  if ((st = check_device())) return st;
+  if (K == 0) return SQ_OK;
+  return cuda_status(
+      launch_fold_norm_weight(gamma, s, K, gamma_s, static_cast<cudaStream_t>(stream)));
+}
+
+int sq_rmsnorm_quant_act(const uint16_t *H, const float *gamma_s, float eps, int64_t M, int64_t K,
+                         int8_t *Xq, float *x_scale, void *stream) {
+  int st = check_mk(M, K);
+  if (st) return st;
+  if (K == 0 || !rmsnorm_quant_supported(K)) return SQ_ERR_UNSUPPORTED_SHAPE;
+  if (!(eps >= 0.0f) || !(eps < 3.4e38f)) return SQ_ERR_INVALID_ARG;
+  if (M > 0 && (!ptr_ok(H) || !ptr_ok(gamma_s) || !ptr_ok(Xq) || !ptr_ok(x_scale)))
+    return SQ_ERR_INVALID_ARG;
+  if ((st = check_device())) return st;
+  return cuda_status(launch_rmsnorm_quant(H, gamma_s, eps, M, K, Xq, x_scale,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 size_t sq_linear_lora_workspace_size(int64_t M, int64_t R) { return workspace_bytes(M, R); }
 
 static int linear_common(const int8_t *Xq, const float *x_scale, const int8_t *Wq,

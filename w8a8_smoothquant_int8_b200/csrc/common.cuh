@@ -56,6 +56,11 @@ cudaError_t launch_static_act_scale(const float *a, const float *s, int64_t K, f
 cudaError_t launch_quant_act_static(const void *X, int dtype, const float *s, const float *scale,
                                     int64_t M, int64_t K, int8_t *Xq, float *x_scale,
                                     unsigned long long *clip_count, cudaStream_t st);
+cudaError_t launch_fold_norm_weight(const float *gamma, const float *s, int64_t K, float *gamma_s,
+                                    cudaStream_t st);
+bool rmsnorm_quant_supported(int64_t K);
+cudaError_t launch_rmsnorm_quant(const uint16_t *H, const float *gamma_s, float eps, int64_t M,
+                                 int64_t K, int8_t *Xq, float *x_scale, cudaStream_t st);
 cudaError_t launch_quantize_weight(const uint16_t *W, const float *s, int64_t N, int64_t K,
                                    int8_t *Wq, float *w_scale, cudaStream_t st);
 cudaError_t launch_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s, int64_t r,

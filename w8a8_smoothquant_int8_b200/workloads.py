@@ -223,6 +223,13 @@ def make_workload(spec, seed: Optional[int] = None, M: Optional[int] = None) -> 
     return Workload(spec, seed, X, X_cal, W, adapters, seg_offsets, seg_adapter, spec.alpha)
 
 
+def norm_gamma(K: int, seed: int) -> np.ndarray:
+    """Weight of an RMS normalization in front of the layer, f32 [K]:
+    1 + 0.1 * N(0, 1), drawn from its own seeded stream."""
+    rng = np.random.default_rng(np.random.PCG64(seed + 7777))
+    return (1.0 + 0.1 * rng.standard_normal(K)).astype(np.float32)
+
+
 def row_adapter(seg_offsets: np.ndarray, seg_adapter: np.ndarray, M: int, n_adapters: int) -> np.ndarray:
     """Adapter index per token (-1 = none) implied by a segment table (layout helper)."""
     out = np.full(M, -1, np.int64)
