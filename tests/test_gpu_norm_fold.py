@@ -9,6 +9,8 @@ most 1e-4 of the rows may differ, each by at most one code step and two ulps
 of x_scale.  Through the linear layer Y stays within the 1e-2 bar.
 """
 
+import math
+
 import numpy as np
 import pytest
 
@@ -82,3 +84,137 @@ def test_norm_fold_through_the_linear_layer():
     ref = oracle.linear_lora_rows(Xq, xs, P.Wq, P.w_scale, P.A_s, P.B_s, wl.seg_offsets,
                                   wl.seg_adapter, rows, want=("Y",))["Y"]
     assert rel_err(g.Y_f32()[rows], ref) <= 1e-2
+
+
+def _assert_parity(H, gamma_s_host, eps, gs_dev=None):
+    """Codes and scales of the GPU kernel against the oracle, same tolerance
+    as above (rows whose fp64 sum of squares is inexact may differ by one)."""
+    import torch
+    import w8a8_smoothquant_int8_b200 as sq
+    from tests.gpu_pipeline import to_dev
+    M, K = H.shape
+    Xq = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    xs = torch.empty(M, dtype=torch.float32, device="cuda")
+    sq.sq_rmsnorm_quant_act(to_dev(H), to_dev(gamma_s_host), eps, Xq, xs)
+    Xq, xs = Xq.cpu().numpy(), xs.cpu().numpy()
+    Xq_ref, xs_ref = oracle.rmsnorm_quant_act(H, gamma_s_host, eps)
+    bad = np.nonzero((xs.view(np.uint32) != xs_ref.view(np.uint32)) | (Xq != Xq_ref).any(1))[0]
+    assert len(bad) <= max(1, int(1e-4 * M)), (bad[:10], xs[bad[:3]], xs_ref[bad[:3]])
+    for i in bad:
+        assert np.abs(Xq[i].astype(np.int64) - Xq_ref[i]).max() <= 1
+        assert abs(int(xs[i].view(np.int32)) - int(xs_ref[i].view(np.int32))) <= 2
+
+
+def _rows(M, K, seed, scale_exp=0.0):
+    # N(0, 1) entries, a log-normal magnitude per row and a few outlier
+    # channels (x20), as bf16
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((M, K)) * np.exp(rng.standard_normal((M, 1)))
+    X[:, rng.choice(K, max(1, K // 256), replace=False)] *= 20.0
+    return wk.f32_to_bf16_bits((X * 2.0 ** scale_exp).astype(np.float32))
+
+
+# every team shape of the streaming kernel (rows of 2 to 2048 16-byte
+# vectors), the block-per-row kernel beyond, ragged row counts and grids with
+# fewer rows than blocks
+@pytest.mark.parametrize("K,M", [(16, 37), (1024, 300), (1040, 129), (2048, 300), (4096, 1),
+                                 (4096, 517), (8192, 300), (14336, 3), (14336, 261),
+                                 (16384, 200), (16400, 70), (32768, 40)])
+def test_norm_quant_shapes(K, M):
+    H = _rows(M, K, seed=K + M)
+    gs = wk.norm_gamma(K, K) / np.float32(1.5)
+    _assert_parity(H, gs.astype(np.float32), EPS)
+
+
+@pytest.mark.parametrize("K", [256, 4096, 14336])
+def test_norm_quant_range_edges(K):
+    # rows whose mean square leaves [2^-100, 2^100] (tiny and huge values
+    # with eps = 0) take the correctly rounded square root and division; a
+    # huge eps puts the row maximum below 2^-60 (IEEE divisions per element);
+    # single-element rows give codes of +-127; an all-zero row with eps = 0
+    # gives r = inf, xt = NaN and codes 0
+    gs = wk.norm_gamma(K, 3).astype(np.float32)
+    for exp, eps in [(-60.0, 0.0), (60.0, 0.0), (0.0, 2.0 ** 126), (-20.0, 2.0 ** 126),
+                     (-30.0, 1e-6)]:
+        _assert_parity(_rows(9, K, seed=int(exp) + 100, scale_exp=exp), gs, eps)
+    H = np.zeros((3, K), np.uint16)
+    H[0, 5] = wk.f32_to_bf16_bits(np.array([-3.0], np.float32))[0]
+    H[1, K - 1] = wk.f32_to_bf16_bits(np.array([2.0 ** -70], np.float32))[0]
+    _assert_parity(H, gs, 0.0)
+
+
+def _bf16_floor_sqrt(R):
+    """Largest bf16 value h with h*h <= R (R a positive Fraction), as
+    (significand m in [128, 255], exponent e): h = m * 2^e."""
+    from fractions import Fraction
+    e = (R.numerator.bit_length() - R.denominator.bit_length()) // 2 - 8
+    while True:
+        x = R / Fraction(2) ** (2 * e)
+        m = math.isqrt(x.numerator // x.denominator)
+        if m < 128:
+            e -= 1
+        elif m > 255:
+            e += 1
+        else:
+            return m, e
+
+
+def _midpoint_row(K, f, delta_exp, sign):
+    """A bf16 row and an eps whose r = 1/sqrt(t) lies at (1 + sign*2^delta_exp)
+    times the point halfway between the float f and the next float up (t
+    from the oracle's fp64 steps).  eps carries t's leading bits; a few
+    squares whose fp64 sum is exact in any order supply the rest."""
+    from fractions import Fraction
+    f32 = np.float32(f)
+    mid = (Fraction(float(f32)) + Fraction(float(np.nextafter(f32, np.float32(np.inf))))) / 2
+    target = mid * (1 + sign * Fraction(2) ** delta_exp) if delta_exp is not None else mid
+    T = 1 / (target * target)
+    eps = np.float32(float(T))
+    while Fraction(float(eps)) > T:
+        eps = np.nextafter(eps, np.float32(0))
+    R = (T - Fraction(float(eps))) * K
+    terms = []
+    for _ in range(4):
+        if R <= 0:
+            break
+        m, e = _bf16_floor_sqrt(R)
+        # keep the squares' sum within 53 bits from the smallest's last bit
+        trial = terms + [(m, e)]
+        emin = min(2 * ee for _, ee in trial)
+        total = sum(mm * mm << (2 * ee - emin) for mm, ee in trial)
+        if total.bit_length() > 53:
+            break
+        terms = trial
+        R -= Fraction(m * m) * Fraction(2) ** (2 * e)
+    vals = np.array([m * 2.0 ** e for m, e in terms], np.float32)
+    H = np.zeros(K, np.uint16)
+    H[np.arange(len(vals)) * (K // max(1, len(vals))) % K] = wk.f32_to_bf16_bits(vals)
+    # the oracle's t and the distance of 1/sqrt(t) from the midpoint
+    ss = 0.0
+    for v in wk.bf16_bits_to_f32(H).astype(np.float64):
+        ss += v * v
+    t = ss / K + float(eps)
+    q = 1 / (Fraction(t) * mid * mid)  # (r / mid)^2
+    return H, float(eps), abs(float(q - 1)) / 2
+
+
+def test_norm_factor_near_float_midpoints():
+    # r_i = RN32(RN64(1/RN64(sqrt(t)))) when 1/sqrt(t) sits almost exactly
+    # halfway between two floats: within 2^-46 the kernel takes the correctly
+    # rounded square root and division; at 2^-44 its Newton estimate decides
+    # (it is within 2^-51 of the double-rounded value)
+    for K in (16, 4096, 14336):
+        gs = np.ones(K, np.float32)
+        rows, epss = [], []
+        for f in (1.0 + 2.0 ** -20, 1.2345, 0.777, 3.5, 0.0123):
+            for delta_exp, sign in [(None, 0), (-50, 1), (-50, -1), (-44, 1), (-44, -1)]:
+                H, eps, dist = _midpoint_row(K, f, delta_exp, sign)
+                if delta_exp is None or delta_exp <= -48:
+                    assert dist < 2.0 ** -47, (K, f, delta_exp, dist)
+                else:
+                    assert 2.0 ** -45 < dist < 2.0 ** -43, (K, f, delta_exp, dist)
+                rows.append(H)
+                epss.append(eps)
+        # one call per eps (eps is a scalar of the call)
+        for H, eps in zip(rows, epss):
+            _assert_parity(H[None, :], gs, eps)
