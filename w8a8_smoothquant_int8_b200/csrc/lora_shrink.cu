@@ -193,6 +193,9 @@ __global__ void __launch_bounds__(kShrinkThreads) lora_shrink_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
   const int rg = warp / kKS, ks = warp % kKS;
   const int64_t row0 = (static_cast<int64_t>(blockIdx.x) * kRG + rg) * 16;
+  // everything this grid reads may come from the preceding kernel (a no-op
+  // unless the grid is launched as a programmatic dependent)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // adapter, column offset and rank of each of the 16 rows of the group
   if (ks == 0 && lane < 16) {
@@ -213,16 +216,18 @@ __global__ void __launch_bounds__(kShrinkThreads) lora_shrink_kernel(
   }
   __syncthreads();
   if (row0 >= M) return;  // whole row group; only group barriers follow
-  // the codes and scales come from the preceding kernel (a no-op unless this
-  // grid is launched as a programmatic dependent)
-  asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // zero both planes for the group's rows, and write the group's mask word
+  // zero both planes where the group's rows get no value below (outside the
+  // row's adapter columns [off, off + rank rounded up to 16); the whole row
+  // for a token without adapter), and write the group's mask word
   {
-    const int64_t nrows = (M - row0 < 16) ? (M - row0) : 16;
-    const int64_t words = nrows * R / 8;  // 16-byte words (R % 16 == 0)
+    const int nrows = static_cast<int>((M - row0 < 16) ? (M - row0) : 16);
+    const int wpr = static_cast<int>(R / 8);  // 16-byte words per row (R % 16 == 0)
     const int tid = ks * 32 + lane;
-    for (int64_t w = tid; w < words; w += kKS * 32) {
+    for (int w = tid; w < nrows * wpr; w += kKS * 32) {
+      const int r = w / wpr, col = (w - r * wpr) * 8;
+      const int a = s_ad[rg][r], off = s_off[rg][r], rpad = (s_rank[rg][r] + 15) & ~15;
+      if (a >= 0 && col >= off && col < off + rpad) continue;
       reinterpret_cast<uint4 *>(T_hi + row0 * R)[w] = make_uint4(0, 0, 0, 0);
       reinterpret_cast<uint4 *>(T_lo + row0 * R)[w] = make_uint4(0, 0, 0, 0);
     }
@@ -318,10 +323,13 @@ static cudaError_t launch_lora_shrink_t(const void *X, const float *x_scale, int
                                         int64_t S, uint16_t *T_hi, uint16_t *T_lo,
                                         unsigned long long *mask, cudaStream_t st) {
   const int64_t row_tiles = (M + 15) / 16;
-  // widest row grouping that still leaves about two blocks per SM.  Launched
-  // in plain stream order: as a programmatic dependent of the quantizer its
-  // blocks were placed worse on the large workloads (measured); the fused
-  // GEMM that follows is launched as its dependent instead.
+  // widest row grouping that still leaves about two blocks per SM.  A grid
+  // of one wave is launched as a programmatic dependent of the preceding
+  // kernel (its blocks wait at the start for that kernel's results, so the
+  // launch gap overlaps the quantizer's tail); larger grids in plain stream
+  // order: as dependents their blocks were placed worse on the large
+  // workloads (measured).  The fused GEMM that follows is launched as the
+  // shrink's dependent.
   const unsigned g1 = static_cast<unsigned>(row_tiles);
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kShrinkThreads, 1, 1);
@@ -348,6 +356,13 @@ static cudaError_t launch_lora_shrink_t(const void *X, const float *x_scale, int
                               T_hi, T_lo, mask);
   }
   cfg.gridDim = dim3(g1, 1, 1);
+  cudaLaunchAttribute attr[1];
+  if (g1 <= static_cast<unsigned>(sm_count_of_current_device())) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
   return cudaLaunchKernelEx(&cfg, lora_shrink_kernel<1, kRaw>, X, x_scale, M, K, A_pack,
                             lora_offset, lora_rank, n_adapters, R, seg_offsets, seg_adapter, S,
                             T_hi, T_lo, mask);
