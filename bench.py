@@ -42,6 +42,11 @@ if ROOT not in sys.path:
 from w8a8_smoothquant_int8_b200 import workloads as wk  # noqa: E402
 
 GEMM_EVENT_EVERY = 8  # timed steps per step that also times the GEMM alone
+# nominal figures, reported beside the measured denominators for context:
+# dense int8 tensor-core ops per SM per clock (4.5 POPS over 148 SMs near
+# 1.9 GHz) and the HBM3e bandwidth of the part
+NOMINAL_INT8_OPS_PER_SM_CLK = 16384
+NOMINAL_HBM_GBS = 8000.0
 
 METRIC = "W8A8+LoRA linear INT8 TOPS & tokens/s; % of INT8 tensor peak / HBM roofline"
 DEFAULT_WORKLOAD = "llama3_8b_qkv_m2048_k4096_n6144"
@@ -449,13 +454,20 @@ def run_ours(args):
         roofline = {"bound": "hbm", "kernel": "decode_shrink_kernel + decode_gemm_kernel",
                     "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                     "peak_source": f"{peak_kind}: copy bandwidth {hbm} GB/s",
+                    "frac_of_nominal": gbs / NOMINAL_HBM_GBS,
                     "layer_us": gemm_avg_s * 1e6, "traffic": None,
                     "traffic_unit": "bytes per launch (ncu dram read+write)",
                     "algorithmic_bytes": nbytes}
     else:
+        # context: the nominal dense int8 rate at the SM clock sampled under load
+        sm_mhz = (clocks or {}).get("sm_mhz") or 0.0
+        n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+        clk_peak = n_sm * NOMINAL_INT8_OPS_PER_SM_CLK * sm_mhz * 1e6 / 1e12
         roofline = {"bound": "tensor", "kernel": "w8a8_lora_gemm_kernel", "achieved": gemm_tops,
                     "peak": int8_peak, "unit": "TOPS", "frac": gemm_tops / int8_peak,
                     "peak_source": f"{peak_kind}: 2 x bf16 burst {peaks['bf16_tflops']} TFLOP/s",
+                    "clock_normalized_peak": clk_peak or None,
+                    "frac_of_clock_normalized": (gemm_tops / clk_peak) if clk_peak else None,
                     "gemm_us": gemm_avg_s * 1e6, "traffic": gemm_traffic(wl.spec.name),
                     "traffic_unit": "bytes per launch (ncu dram read+write)",
                     "algorithmic_ops": ops_step}
