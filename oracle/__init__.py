@@ -59,6 +59,7 @@ def lib():
             "sqo_static_act_scale": ([P, P, I64], F),
             "sqo_fold_norm_weight": ([P, P, I64, P], None),
             "sqo_rmsnorm_quant_act": ([P, P, F, I64, I64, P, P], None),
+            "sqo_sum_squares_bf16": ([P, I64], ctypes.c_double),
             "sqo_quant_act_static": ([P, I32, P, F, I64, I64, P, P], I64),
             "sqo_gemm_rows": ([P, P, I64, I64, I64, P, I64, P], None),
             "sqo_gemm_pairs": ([P, P, I64, P, P, I64, P], None),
@@ -178,6 +179,12 @@ def fold_norm_weight(gamma: np.ndarray, s: np.ndarray) -> np.ndarray:
     out = np.zeros_like(g)
     lib().sqo_fold_norm_weight(_p(g), _p(s), g.shape[0], _p(out))
     return out
+
+
+def sum_squares_bf16(h: np.ndarray) -> float:
+    """Exact sum of the squares of a bf16 row, rounded once to fp64."""
+    h = _c(h, np.uint16).ravel()
+    return float(lib().sqo_sum_squares_bf16(_p(h), h.shape[0]))
 
 
 def rmsnorm_quant_act(H: np.ndarray, gamma_s: np.ndarray, eps: float):

@@ -237,17 +237,69 @@ void sqo_fold_norm_weight(const float *gamma, const float *s, int64_t K, float *
  *   r_i  = RN32( 1 / sqrt( (sum_j h_ij^2) / K + eps ) )   (fp64 inside)
  *   xt   = RN32( RN32(h_ij * r_i) * gamma_s[j] )
  *   x_scale_i = RN32(max_j |xt| / 127),  Xq = clamp(RNE(RN32(xt / x_scale_i)))
- * H [M,K] bf16.  The sum of squares of bf16 values is exact in fp64 whenever
- * a row's squares span less than 2^37 in magnitude; it is summed in order. */
+ * H [M,K] bf16.  The sum of squares is defined as the exact sum of the
+ * (exact) squares of the bf16 values, rounded once to fp64, so it does not
+ * depend on any order of summation (a row's squares can span far more than
+ * the 53 bits of an fp64 sum); the square root and the division are the
+ * correctly rounded fp64 operations. */
+
+/* Sum of the squares of K bf16 values, exact, rounded once to fp64 (nearest,
+ * ties to even).  A finite bf16 value with exponent field E and fraction field
+ * F is m * 2^(max(E,1) - 134) with the integer significand m = F (E == 0) or
+ * 128 + F, so its square is the integer m^2 (< 2^16) times 2^(2*max(E,1) - 268):
+ * the integer m^2 shifted left by 2*max(E,1) - 2 bits in a fixed-point number
+ * whose unit is 2^-266.  That number is kept in 32-bit digits (the largest
+ * square ends below bit 522, and up to 2^20 squares add at most 20 bits), then
+ * its top 53 bits are rounded using the next bit and whether any bit below it
+ * is set.  A row holding an infinity or a NaN gives the fp64 sum of its
+ * squares (inf or NaN). */
+#define SQO_SS_DIGITS 18
+double sqo_sum_squares_bf16(const uint16_t *h, int64_t K) {
+  uint32_t d[SQO_SS_DIGITS];
+  memset(d, 0, sizeof d);
+  for (int64_t j = 0; j < K; ++j) {
+    unsigned E = (h[j] >> 7) & 0xFFu, F = h[j] & 0x7Fu;
+    if (E == 0xFFu) { /* not finite */
+      double s = 0.0;
+      for (int64_t t = 0; t < K; ++t) s += bf16_value(h[t]) * bf16_value(h[t]);
+      return s;
+    }
+    uint64_t m = (E == 0) ? F : (128u + F);
+    if (m == 0) continue;
+    unsigned pos = 2u * (E == 0 ? 1u : E) - 2u; /* bit position of m^2 */
+    /* add (m^2 << pos) digit by digit with carry */
+    uint64_t carry = (m * m) << (pos % 32u); /* < 2^48 */
+    for (unsigned k = pos / 32u; carry != 0 && k < SQO_SS_DIGITS; ++k) {
+      carry += d[k];
+      d[k] = (uint32_t)carry;
+      carry >>= 32;
+    }
+  }
+  int top = -1; /* highest set bit */
+  for (int k = SQO_SS_DIGITS - 1; k >= 0 && top < 0; --k)
+    for (int b = 31; b >= 0; --b)
+      if ((d[k] >> b) & 1u) { top = 32 * k + b; break; }
+  if (top < 0) return 0.0;
+#define SQO_BIT(p) ((p) >= 0 ? (int)((d[(p) / 32] >> ((p) % 32)) & 1u) : 0)
+  /* the 53 bits from `top` down, as an integer */
+  uint64_t sig = 0;
+  for (int p = top; p > top - 53; --p) sig = (sig << 1) | (uint64_t)SQO_BIT(p);
+  int lsb = top - 52; /* weight 2^(lsb - 266) of the last kept bit */
+  if (lsb > 0) {
+    int round = SQO_BIT(lsb - 1), sticky = 0;
+    for (int p = lsb - 2; p >= 0; --p) sticky |= SQO_BIT(p);
+    if (round && (sticky || (sig & 1u))) sig += 1; /* may reach 2^53: still exact */
+  }
+#undef SQO_BIT
+  return ldexp((double)sig, lsb - 266);
+}
+
 void sqo_rmsnorm_quant_act(const uint16_t *H, const float *gamma_s, float eps, int64_t M,
                            int64_t K, int8_t *Xq, float *x_scale) {
 #pragma omp parallel for schedule(static)
   for (int64_t i = 0; i < M; ++i) {
-    double ss = 0.0;
-    for (int64_t j = 0; j < K; ++j) {
-      double h = bf16_value(H[i * K + j]);
-      ss += h * h;
-    }
+    /* the sum of squares is the exact one, rounded once to fp64 */
+    double ss = sqo_sum_squares_bf16(H + i * K, K);
     float r = rn32(1.0 / sqrt(ss / (double)K + (double)eps));
     double amax = 0.0;
     for (int64_t j = 0; j < K; ++j) {

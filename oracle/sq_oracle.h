@@ -34,6 +34,7 @@ float sqo_static_act_scale(const float *act_absmax, const float *s, int64_t K);
 int64_t sqo_quant_act_static(const void *X, int dtype, const float *s, float scale, int64_t M,
                              int64_t K, int8_t *Xq, float *x_scale);
 void sqo_fold_norm_weight(const float *gamma, const float *s, int64_t K, float *gamma_s);
+double sqo_sum_squares_bf16(const uint16_t *h, int64_t K);
 void sqo_rmsnorm_quant_act(const uint16_t *H, const float *gamma_s, float eps, int64_t M,
                            int64_t K, int8_t *Xq, float *x_scale);
 void sqo_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s, int64_t r,
