@@ -10,21 +10,24 @@ namespace sq {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[SQ_NOALLOC_SCRATCH_BYTES];
 
 // Device address of g_noalloc_scratch on each device, looked up on the first
-// call made with that device current.  In host code the array's name is only
-// a host-side stand-in, never a device address.
-static void *g_noalloc_scratch_addr[64] = {nullptr};
+// call made with that device current (std::atomic: host threads may call
+// concurrently; two that find the slot empty store the same address).  In
+// host code the array's name is only a host-side stand-in, never a device
+// address.  After cudaDeviceReset of a device the cached address is stale:
+// the library must not be used on that device again.
+static std::atomic<void *> g_noalloc_scratch_addr[kMaxDevices];
 
 static int noalloc_scratch(void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SQ_ERR_CUDA;
-  if (dev < 0 || dev >= 64) return SQ_ERR_UNSUPPORTED_DEVICE;
-  if (!g_noalloc_scratch_addr[dev]) {
-    void *p = nullptr;
+  if (dev < 0 || dev >= kMaxDevices) return SQ_ERR_UNSUPPORTED_DEVICE;
+  void *p = g_noalloc_scratch_addr[dev].load(std::memory_order_acquire);
+  if (!p) {
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return SQ_ERR_CUDA;
-    g_noalloc_scratch_addr[dev] = p;
+    g_noalloc_scratch_addr[dev].store(p, std::memory_order_release);
   }
-  *out = g_noalloc_scratch_addr[dev];
+  *out = p;
   return SQ_OK;
 }
 
@@ -37,14 +40,15 @@ extern "C" int sq_linear_lora_noalloc(const int8_t *Xq, const float *x_scale, co
                                       int n_adapters, int64_t R, const int32_t *seg_offsets,
                                       const int32_t *seg_adapter, int64_t S, uint16_t *Y,
                                       void *stream) {
-  if (M < 0 || R < 0) return SQ_ERR_INVALID_ARG;
-  if (sq_linear_lora_workspace_size(M, R) > SQ_NOALLOC_SCRATCH_BYTES) return SQ_ERR_WORKSPACE;
+  // the scratch's address needs the library's module on this device
   int st = sq_device_supported_current();
   if (st) return st;
   void *scratch = nullptr;
   if ((st = sq::noalloc_scratch(&scratch))) return st;
-  // every byte the kernels read from the scratch is written earlier in the
-  // same call (the tile masks are cleared by the launch sequence itself)
+  // sq_linear_lora checks everything else, the scratch's size as it checks a
+  // caller's workspace (after the shapes, and only when an adapter is in
+  // play).  Every byte the kernels read from the scratch is written earlier
+  // in the same call (the tile masks are cleared by the launch sequence).
   return sq_linear_lora(Xq, x_scale, Wq, w_scale, M, N, K, A_pack, B_pack, lora_offset, lora_rank,
                         n_adapters, R, seg_offsets, seg_adapter, S, Y, scratch,
                         SQ_NOALLOC_SCRATCH_BYTES, stream);
