@@ -188,13 +188,14 @@ int sq_fold_norm_weight(const float *gamma, const float *s, int64_t K, float *ga
                         void *stream);
 
 /* RMS normalization with the folded weight fused with Step 6 (per token):
- *   r_i = RN32(1 / sqrt(sum_j H[i,j]^2 / K + eps))  (fp64 sum of the exact
- *         squares, correctly rounded sqrt and division),
+ *   r_i = RN32(1 / sqrt(ss_i / K + eps))  with ss_i the exact sum of the
+ *         squares of the row, rounded once to fp64; the division by K, the
+ *         + eps, the square root and the reciprocal are correctly rounded
+ *         fp64 operations,
  *   xt = RN(RN(H[i,j] * r_i) * gamma_s[j]);  x_scale_i = RN(max_j |xt| / 127);
  *   Xq = clamp(round_half_even(RN(xt / x_scale_i)), -128, 127).
- * H [M,K] bf16 (the layer's pre-normalization input), device.  Bit-exact
- * while a row's squares span less than 2^37 (the fp64 sum is then exact, so
- * its order does not matter).  K % 16 == 0 and K <= 32768, else
+ * H [M,K] bf16 (the layer's pre-normalization input), device.  Bit-exact for
+ * every finite row.  K % 16 == 0 and K <= 32768, else
  * SQ_ERR_UNSUPPORTED_SHAPE; eps >= 0. */
 int sq_rmsnorm_quant_act(const uint16_t *H, const float *gamma_s, float eps, int64_t M, int64_t K,
                          int8_t *Xq, float *x_scale, void *stream);
@@ -236,12 +237,17 @@ int sq_linear_lora(const int8_t *Xq, const float *x_scale, const int8_t *Wq,
  * The scratch is one static device array of SQ_NOALLOC_SCRATCH_BYTES (16 MiB)
  * that every GPU loading the library holds until the process exits; a call
  * whose sq_linear_lora_workspace_size(M, R) exceeds it returns
- * SQ_ERR_WORKSPACE.  The first call on each device looks up the array's
- * device address (cudaGetSymbolAddress), so make that first call before any
- * stream capture.  Each device has its own copy of the array and every call
- * on that device uses it, keeping what the last call left there: calls that
- * overlap on one GPU (for example on two streams) race, so serialize them.
- * Other arguments, results and errors as sq_linear_lora.  Allocates nothing. */
+ * SQ_ERR_WORKSPACE (checked after the shapes, and only when an adapter is in
+ * play, as sq_linear_lora checks a workspace).  The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress), so make that
+ * first call before any stream capture; on a device that is not compute
+ * capability 10.0 every call returns SQ_ERR_UNSUPPORTED_DEVICE before its
+ * arguments are looked at.  Each device has its own copy of the array and
+ * every call on that device uses it, keeping what the last call left there:
+ * calls that overlap on one GPU (for example on two streams) race, so
+ * serialize them.  After cudaDeviceReset of a device the library must not be
+ * used on it again.  Other arguments, results and errors as sq_linear_lora.
+ * Allocates nothing. */
 int sq_linear_lora_noalloc(const int8_t *Xq, const float *x_scale, const int8_t *Wq,
                            const float *w_scale, int64_t M, int64_t N, int64_t K,
                            const uint16_t *A_pack, const uint16_t *B_pack,
@@ -283,6 +289,25 @@ size_t sq_alpha_error_workspace_size(int64_t M, int64_t N, int64_t K);
 int sq_alpha_output_error(const void *X, int x_dtype, const uint16_t *W, int64_t M, int64_t N,
                           int64_t K, float alpha, double *err, void *workspace,
                           size_t workspace_bytes, void *stream);
+
+/* Largest number of alpha values of one sq_alpha_sweep. */
+#define SQ_ALPHA_SWEEP_MAX 64
+
+/* The per-layer choice of alpha by calibration error ("SmoothQuant"
+ * explainer, "Variants and related ideas": pick alpha layer by layer by the
+ * output error on calibration data; "Reading the diagnostics": a sharp
+ * minimum suggests a good choice).  For each of the n values alphas[t] (host
+ * array, 1 <= n <= SQ_ALPHA_SWEEP_MAX, each in [0, 1]) the two sums of
+ * sq_alpha_output_error go to err[2t], err[2t+1]; then
+ *   rel[t] = err[2t] / err[2t+1]   (IEEE fp64 division; 0 if err[2t+1] == 0)
+ * and *best = the alpha with the smallest rel (the first one on ties).
+ * err [2n] double, rel [n] double, best one float: device memory, written
+ * on the stream (no host synchronization).  X, W, shapes and workspace as for
+ * sq_alpha_output_error; errors as there, plus SQ_ERR_INVALID_ARG for n or
+ * an alpha out of range. */
+int sq_alpha_sweep(const void *X, int x_dtype, const uint16_t *W, int64_t M, int64_t N, int64_t K,
+                   const float *alphas, int n, double *err, double *rel, float *best,
+                   void *workspace, size_t workspace_bytes, void *stream);
 
 /* ---------------------------------------------------------------------------
  * Raw-input reading of the LoRA path ("[Feature]: LoRA support for W8A8
