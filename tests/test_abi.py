@@ -172,6 +172,24 @@ def test_alpha_error_entry_validation(lib):
     assert f(A, 1, A, 64, 128, 256, 0.5, A, A, wsz, None) in (CUDA, DEVICE)
 
 
+def test_alpha_sweep_entry_validation(lib):
+    wsz = lib.sq_alpha_error_workspace_size(64, 128, 256)
+    f = lib.sq_alpha_sweep
+
+    def alphas(*v):
+        return (ctypes.c_float * max(1, len(v)))(*v)
+
+    good = alphas(0.0, 0.5, 1.0)
+    assert f(A, 1, A, 64, 128, 256, good, 0, A, A, A, A, wsz, None) == INVALID    # no alpha
+    assert f(A, 1, A, 64, 128, 256, alphas(*([0.5] * 65)), 65, A, A, A, A, wsz, None) == INVALID
+    assert f(A, 1, A, 64, 128, 256, alphas(0.5, -0.1), 2, A, A, A, A, wsz, None) == INVALID
+    assert f(A, 1, A, 64, 128, 256, None, 3, A, A, A, A, wsz, None) == INVALID
+    assert f(A, 1, A, 64, 100, 256, good, 3, A, A, A, A, wsz, None) == SHAPE      # N % 16
+    assert f(A, 1, A, 64, 128, 256, good, 3, A + 4, A, A, A, wsz, None) == INVALID  # err align
+    assert f(A, 1, A, 64, 128, 256, good, 3, A, A, A, A, wsz - 1, None) == WORKSPACE
+    assert f(A, 1, A, 64, 128, 256, good, 3, A, A, A, A, wsz, None) in (CUDA, DEVICE)
+
+
 def test_norm_fold_entry_validation(lib):
     assert lib.sq_fold_norm_weight(A, A, 1000, A, None) == SHAPE
     assert lib.sq_fold_norm_weight(A + 4, A, 64, A, None) == INVALID

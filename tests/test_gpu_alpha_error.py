@@ -71,3 +71,29 @@ def test_alpha_error_raw_sums():
     sq.sq_alpha_output_error(X, W, 0.5, err, ws)
     e2, r2 = err.cpu().numpy()
     assert abs(e2 - e) <= 1e-9 * e and abs(r2 - r) <= 1e-9 * r
+
+
+def test_alpha_sweep_entry_outputs():
+    # the C entry's device outputs: the sums per alpha equal single calls of
+    # sq_alpha_output_error, rel is their ratio, best the first minimum
+    import torch
+    import w8a8_smoothquant_int8_b200 as sq
+    from tests.gpu_pipeline import to_dev
+    wl = wk.make_workload("parity_ragged")
+    X, W = to_dev(wl.X_cal), to_dev(wl.W)
+    M, K, N = X.shape[0], X.shape[1], W.shape[0]
+    ws = torch.empty(sq.sq_alpha_error_workspace_size(M, N, K), dtype=torch.uint8, device="cuda")
+    alphas = [0.5, 0.25, 0.5, 0.75]
+    err = torch.empty(2 * len(alphas), dtype=torch.float64, device="cuda")
+    rel = torch.empty(len(alphas), dtype=torch.float64, device="cuda")
+    best = torch.empty(1, dtype=torch.float32, device="cuda")
+    sq.sq_alpha_sweep(X, W, alphas, err, rel, best, ws)
+    e = err.cpu().numpy().reshape(-1, 2)
+    r = rel.cpu().numpy()
+    one = torch.empty(2, dtype=torch.float64, device="cuda")
+    for t, a in enumerate(alphas):
+        sq.sq_alpha_output_error(X, W, a, one, ws)
+        # (the sums are fp64 atomics: equal up to their order of addition)
+        assert np.allclose(one.cpu().numpy(), e[t], rtol=1e-9, atol=0)
+        assert r[t] == e[t, 0] / e[t, 1]
+    assert float(best.cpu()[0]) == alphas[int(np.argmin(r))]

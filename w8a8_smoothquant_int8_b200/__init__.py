@@ -24,7 +24,7 @@ __all__ = [
     "sq_linear_lora_workspace_size", "sq_linear_lora", "sq_linear_lora_noalloc", "sq_gemm_i32",
     "sq_lora_delta", "sq_lora_t_workspace_size", "sq_lora_shrink_raw", "sq_linear_lora_from_t",
     "sq_lora_delta_from_t", "sq_static_act_scale", "sq_quant_act_static",
-    "sq_alpha_error_workspace_size", "sq_alpha_output_error", "alpha_sweep",
+    "sq_alpha_error_workspace_size", "sq_alpha_output_error", "sq_alpha_sweep", "alpha_sweep",
     "sq_fold_norm_weight", "sq_rmsnorm_quant_act",
 ]
 
@@ -274,22 +274,33 @@ def sq_alpha_output_error(X, W, alpha: float, err, workspace, stream=None) -> No
            "sq_alpha_output_error")
 
 
+def sq_alpha_sweep(X, W, alphas: Sequence[float], err, rel, best, workspace, stream=None) -> None:
+    """err [2n], rel [n] (float64) and best [1] (float32) device tensors from
+    one sweep over the host list `alphas` (see sq_alpha_sweep in the header)."""
+    M, K = X.shape
+    N = W.shape[0]
+    arr = (ctypes.c_float * max(1, len(alphas)))(*[float(a) for a in alphas])
+    wp, wb = _ws(workspace)
+    _check(_lib().sq_alpha_sweep(_ptr(X), _xdtype(X), _ptr(W), M, N, K, arr, len(alphas),
+                                 _ptr(err), _ptr(rel), _ptr(best), wp, wb, _stream(stream)),
+           "sq_alpha_sweep")
+
+
 def alpha_sweep(X_cal, W, alphas: Sequence[float], stream=None):
     """Per-layer migration strength by calibration error: the relative
-    squared output error ||Y - X W^T||^2 / ||X W^T||^2 of the W8A8 layer for
-    each alpha, on the calibration tokens.  Returns (errors, best alpha)."""
+    squared output error of the W8A8 layer for each alpha on the calibration
+    tokens, and the alpha with the smallest (sq_alpha_sweep).  Returns
+    (errors as a list, best alpha)."""
     import torch
     M, K = X_cal.shape
     N = W.shape[0]
-    ws = torch.empty(max(sq_alpha_error_workspace_size(M, N, K), 256), dtype=torch.uint8,
-                     device=X_cal.device)
-    err = torch.empty((len(alphas), 2), dtype=torch.float64, device=X_cal.device)
-    for i, a in enumerate(alphas):
-        sq_alpha_output_error(X_cal, W, a, err[i], ws, stream)
-    e = err.cpu()
-    rel = [float(e[i, 0] / e[i, 1]) if float(e[i, 1]) > 0 else 0.0 for i in range(len(alphas))]
-    best = min(range(len(alphas)), key=lambda i: rel[i]) if alphas else -1
-    return rel, (float(alphas[best]) if best >= 0 else None)
+    dev = X_cal.device
+    ws = torch.empty(max(sq_alpha_error_workspace_size(M, N, K), 256), dtype=torch.uint8, device=dev)
+    err = torch.empty(2 * len(alphas), dtype=torch.float64, device=dev)
+    rel = torch.empty(len(alphas), dtype=torch.float64, device=dev)
+    best = torch.empty(1, dtype=torch.float32, device=dev)
+    sq_alpha_sweep(X_cal, W, alphas, err, rel, best, ws, stream)
+    return rel.cpu().tolist(), float(best.cpu()[0])
 
 
 def sq_lora_t_workspace_size(M: int, R: int) -> int:

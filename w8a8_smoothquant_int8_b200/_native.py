@@ -45,6 +45,7 @@ SIGNATURES = {
     "sq_rmsnorm_quant_act": ([P, P, F32, I64, I64, P, P, P], I32),
     "sq_alpha_error_workspace_size": ([I64, I64, I64], SZ),
     "sq_alpha_output_error": ([P, I32, P, I64, I64, I64, F32, P, P, SZ, P], I32),
+    "sq_alpha_sweep": ([P, I32, P, I64, I64, I64, P, I32, P, P, P, P, SZ, P], I32),
     "sq_static_act_scale": ([P, P, I64, P, P], I32),
     "sq_quant_act_static": ([P, I32, P, P, I64, I64, P, P, P, P], I32),
     "sq_lora_shrink_raw": ([P, I64, I64, P, P, P, I32, I64, P, P, I64, P, SZ, P], I32),

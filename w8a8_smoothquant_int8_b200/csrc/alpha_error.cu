@@ -149,4 +149,44 @@ cudaError_t launch_alpha_error(const void *X, int dtype, const uint16_t *W, int6
   return cudaGetLastError();
 }
 
+// The choice of alpha from the sweep's sums: rel[t] = err[t][0] / err[t][1]
+// (IEEE fp64 division; 0 when the reference energy is 0) and *best = the
+// alpha of the smallest rel, the first one on ties.  One thread: at most
+// kAlphaSweepMax values.
+struct AlphaList {
+  float a[kAlphaSweepMax];
+  int n;
+};
+
+__global__ void alpha_pick_kernel(const double *__restrict__ err, AlphaList al,
+                                  double *__restrict__ rel, float *__restrict__ best) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int bi = 0;
+  double bv = 0.0;
+  for (int t = 0; t < al.n; ++t) {
+    const double den = err[2 * t + 1];
+    const double r = den > 0.0 ? __ddiv_rn(err[2 * t], den) : 0.0;
+    rel[t] = r;
+    if (t == 0 || r < bv) {
+      bv = r;
+      bi = t;
+    }
+  }
+  *best = al.a[bi];
+}
+
+cudaError_t launch_alpha_sweep(const void *X, int dtype, const uint16_t *W, int64_t M, int64_t N,
+                               int64_t K, const float *alphas, int n, double *err, double *rel,
+                               float *best, void *workspace, cudaStream_t st) {
+  AlphaList al;
+  al.n = n;
+  for (int t = 0; t < n; ++t) {
+    al.a[t] = alphas[t];
+    const cudaError_t e = launch_alpha_error(X, dtype, W, M, N, K, alphas[t], err + 2 * t, workspace, st);
+    if (e != cudaSuccess) return e;
+  }
+  alpha_pick_kernel<<<1, 32, 0, st>>>(err, al, rel, best);
+  return cudaGetLastError();
+}
+
 }  // namespace sq

@@ -8,7 +8,7 @@
 
 namespace sq {
 
-static uint64_t g_wait_timeout_ns = 2000000000ull;
+static std::atomic<uint64_t> g_wait_timeout_ns{2000000000ull};
 static cudaEvent_t g_gemm_ev_before = nullptr, g_gemm_ev_after = nullptr;
 uint64_t wait_timeout_ns() { return g_wait_timeout_ns; }
 
@@ -21,16 +21,18 @@ static bool ptr_ok(const void *p) { return p != nullptr && aligned16(p); }
 // Result of sq_device_supported per device, cached: querying the device
 // properties takes far longer than a launch.
 static int check_device() {
-  static int cached[64] = {0};  // 0 = unknown, else status + 1
+  static std::atomic<int> cached[kMaxDevices];  // 0 = unknown, else status + 1
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SQ_ERR_CUDA;
-  if (dev < 0 || dev >= 64) return sq_device_supported(dev);
-  if (cached[dev] == 0) {
-    int st = sq_device_supported(dev);
+  if (dev < 0 || dev >= kMaxDevices) return sq_device_supported(dev);
+  int c = cached[dev].load(std::memory_order_relaxed);
+  if (c == 0) {
+    const int st = sq_device_supported(dev);
     if (st == SQ_ERR_CUDA) return st;
-    cached[dev] = st + 1;
+    c = st + 1;
+    cached[dev].store(c, std::memory_order_relaxed);
   }
-  return cached[dev] - 1;
+  return c - 1;
 }
 
 static int check_mk(int64_t M, int64_t K) {
@@ -408,6 +410,27 @@ int sq_alpha_output_error(const void *X, int x_dtype, const uint16_t *W, int64_t
   if ((st = check_device())) return st;
   return cuda_status(launch_alpha_error(X, x_dtype, W, M, N, K, alpha, err, workspace,
                                         static_cast<cudaStream_t>(stream)));
+}
+
+int sq_alpha_sweep(const void *X, int x_dtype, const uint16_t *W, int64_t M, int64_t N, int64_t K,
+                   const float *alphas, int n, double *err, double *rel, float *best,
+                   void *workspace, size_t workspace_size, void *stream) {
+  int st = check_mk(M, K);
+  if (st) return st;
+  if (x_dtype != SQ_DTYPE_BF16 && x_dtype != SQ_DTYPE_F32) return SQ_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0 || n < 1 || n > SQ_ALPHA_SWEEP_MAX || !alphas)
+    return SQ_ERR_INVALID_ARG;
+  for (int t = 0; t < n; ++t)
+    if (!(alphas[t] >= 0.0f && alphas[t] <= 1.0f)) return SQ_ERR_INVALID_ARG;
+  if (N % 16 != 0) return SQ_ERR_UNSUPPORTED_SHAPE;
+  if (!ptr_ok(X) || !ptr_ok(W) || !aligned_to(err, 8) || !aligned_to(rel, 8) || !aligned_to(best, 4))
+    return SQ_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_size < alpha_error_workspace_bytes(M, N, K))
+    return SQ_ERR_WORKSPACE;
+  if ((st = check_device())) return st;
+  return cuda_status(launch_alpha_sweep(X, x_dtype, W, M, N, K, alphas, n, err, rel, best,
+                                        workspace, static_cast<cudaStream_t>(stream)));
 }
 
 // ---- raw-input reading of the LoRA path ------------------------------------

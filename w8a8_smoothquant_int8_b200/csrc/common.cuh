@@ -1,6 +1,7 @@
 // Shared definitions of the CUDA library (not part of the public ABI).
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -19,18 +20,65 @@ __device__ __forceinline__ void record_device_error(unsigned int code) {
 // Default bound of every device-side spin-wait (ns), settable from the host.
 uint64_t wait_timeout_ns();
 
+// Launch facts are kept per device: a process may drive several GPUs, and
+// kernel attributes and occupancies belong to a device.  The caches are
+// atomics, so host threads may launch concurrently (two threads that find a
+// slot empty both compute the same value).  They hold for the life of the
+// process: after cudaDeviceReset of a device the library must not be used on
+// that device again.
+constexpr int kMaxDevices = 64;
+
+// The current device, or -1 when it cannot be queried or is beyond the caches.
+static inline int current_device_index() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
 // Number of SMs of the current device (cached per device).
 static inline int sm_count_of_current_device() {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int n = 0;
+  static std::atomic<int> cached[kMaxDevices];
+  const int dev = current_device_index();
+  if (dev < 0) return 148;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = n > 0 ? n : 148;
+    n = n > 0 ? n : 148;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
+}
+
+// Sets the dynamic shared-memory opt-in of `kern` to `bytes` once per device;
+// `done` holds one flag per device (one array per kernel).
+template <class Kern>
+static inline cudaError_t ensure_smem_optin(Kern kern, int bytes,
+                                            std::atomic<int> (&done)[kMaxDevices]) {
+  const int dev = current_device_index();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done[dev].store(1, std::memory_order_release);
+  return e;
+}
+
+// Resident blocks per SM of `kern` with `threads` threads and `smem` bytes of
+// dynamic shared memory on the current device, cached per device in
+// cache[dev][slot] (the caller's slot stands for its shared-memory size).
+template <class Kern, int kSlots>
+static inline cudaError_t blocks_per_sm(Kern kern, int threads, size_t smem, int slot,
+                                        std::atomic<int> (&cache)[kMaxDevices][kSlots], int *out) {
+  const int dev = current_device_index();
+  if (dev < 0 || slot < 0 || slot >= kSlots) return cudaErrorInvalidValue;
+  int bps = cache[dev][slot].load(std::memory_order_relaxed);
+  if (bps == 0) {
+    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, kern, threads, smem);
+    if (e != cudaSuccess) return e;
+    bps = bps > 0 ? bps : 1;
+    cache[dev][slot].store(bps, std::memory_order_relaxed);
+  }
+  *out = bps;
+  return cudaSuccess;
 }
 
 // LoRA operands of the fused GEMM: T planes [M,R] bf16 (written by the
@@ -91,6 +139,10 @@ cudaError_t launch_w8a8_gemm(const int8_t *Xq, const int8_t *Wq, const float *x_
                              void *out, const LoraOperands *lora, cudaStream_t st);
 
 size_t alpha_error_workspace_bytes(int64_t M, int64_t N, int64_t K);
+constexpr int kAlphaSweepMax = SQ_ALPHA_SWEEP_MAX;
+cudaError_t launch_alpha_sweep(const void *X, int dtype, const uint16_t *W, int64_t M, int64_t N,
+                               int64_t K, const float *alphas, int n, double *err, double *rel,
+                               float *best, void *workspace, cudaStream_t st);
 cudaError_t launch_alpha_error(const void *X, int dtype, const uint16_t *W, int64_t M, int64_t N,
                                int64_t K, float alpha, double *err, void *workspace,
                                cudaStream_t st);

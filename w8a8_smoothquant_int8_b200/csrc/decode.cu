@@ -1,21 +1,26 @@
 // Small-M (decode) form of the W8A8 + LoRA linear ("SmoothQuant" explainer,
-// Step 7 and "Smaller gain at small batches ... memory-bound"; "[Feature]:
-// LoRA support for W8A8 SmoothQuant", Pitch and Motivation: one adapter per
-// request).  With a few dozen tokens the layer is bound by streaming Wq and
-// the adapters from HBM, so the work is spread over output-channel slices
-// rather than 256x256 tiles:
-//   kernel 1 (shrink)   one warp per (token, K slice): partial sums of
-//                       T[i,:] = x_scale_i * Xq[i,:] A_a^T over the slice,
-//                       written to a scratch table (no atomics: the sums are
-//                       later added in a fixed order); it lets the GEMM grid
-//                       launch at once, so the weight stream overlaps it;
-//   kernel 2 (GEMM + expand), one block per 32 output channels:
-//                       acc = Xq Wq^T with int8 tensor-core MMAs (m16n8k32,
-//                       exact int32) from a TMA-fed ring of Wq tiles; then,
-//                       after the shrink grid has completed (programmatic
-//                       dependent launch: the weight stream starts before the
-//                       shrink finishes), delta = T B_a^T in fp32 and
-//                       Y = bf16(acc*xs*ws + delta).
+// Step 7 and "Limitations": smaller gain at small batches, memory-bound;
+// "[Feature]: LoRA support for W8A8 SmoothQuant", Pitch and Motivation: one
+// adapter per request).  With a few dozen tokens the layer is bound by
+// streaming Wq and the adapters from HBM, so the aim is to keep every SM
+// pulling bytes from the first to the last microsecond:
+//   kernel 1 (shrink)   one block per (token, K slice): the partial sums of
+//                       T[i,:] = Xq[i,:] A_a^T over the slice, every A' row of
+//                       the adapter requested at once; it lets the GEMM grid
+//                       launch at once, so both stream side by side;
+//   kernel 2 (GEMM + expand), CTA pairs (thread-block clusters of two): each
+//                       pair owns a tile of up to 64 output channels and each
+//                       CTA of the pair one half of K, so a CTA streams its
+//                       half of the Wq tile and the matching half of Xq
+//                       through a TMA ring once; acc = Xq Wq^T with int8
+//                       tensor-core MMAs (m16n8k32, exact int32); the two
+//                       halves are added through distributed shared memory;
+//                       the B' rows of the CTA's output channels are
+//                       bulk-copied into shared memory while the weights
+//                       stream; after the shrink grid has completed
+//                       (programmatic dependent launch), T = x_scale * (sum of
+//                       the partials in a fixed order) and
+//                       Y = bf16(acc*xs*ws + T B_a^T).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -24,17 +29,105 @@
 
 namespace sq {
 
-constexpr int kDecMaxM = 64;       // token rows handled by this form
-constexpr int kDecMaxRank = 256;   // largest adapter rank (the library-wide limit)
-constexpr int kDecKSplit = 16;     // K slices of the shrink
-constexpr int kDecCols = 32;       // output channels per GEMM block
-constexpr int kDecThreads = 256;
+constexpr int kDecMaxM = 64;            // token rows handled by this form
+constexpr int kDecMaxRank = 256;        // largest adapter rank (the library-wide limit)
+constexpr int kDecTable = 256;          // adapter table entries staged in shared memory
+constexpr int kDecShrinkThreads = 256;
+constexpr int kDecShrinkSplitMax = 8;   // K slices of the shrink, at most
+constexpr int kDecShrinkSpan = 2048;    // K elements a shrink block covers per pass
+
+__device__ __forceinline__ void group_bar(int id, int nthr) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthr) : "memory");
+}
 
 // ---------------------------------------------------------------------------
-// kernel 1: shrink partials.  part[(i * kDecKSplit + ks) * kDecMaxRank + j]
+// Adapter of each token.  Token i belongs to the first segment s with
+// seg_offsets[s] <= i < seg_offsets[s+1] and takes adapter seg_adapter[s]
+// (-1: none).  Every segment is examined by one thread of the group, all in
+// one round of loads, and the smallest covering s wins through a
+// shared-memory minimum over (s, adapter) keys; the adapters' column offsets
+// and ranks are staged in the same round when there are at most kDecTable of
+// them.  Results for tokens [t0, t0 + nt): off[k], rank[k] (rank 0: no
+// adapter; an index or an offset/rank out of range is recorded as
+// SQ_ERR_BAD_SEGMENTS and the token gets no adapter).  `bar_id` names a
+// barrier over the group's `nthr` threads.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kDecThreads, 1) decode_shrink_kernel(
-    const int8_t *__restrict__ Xq, const float *__restrict__ x_scale, int64_t M, int64_t K,
+struct DecodeTables {
+  unsigned long long best[kDecMaxM];
+  int ad_off[kDecTable];
+  int ad_rank[kDecTable];
+};
+
+__device__ void decode_lookup(const int32_t *__restrict__ seg_offsets,
+                              const int32_t *__restrict__ seg_adapter, int64_t S,
+                              const int32_t *__restrict__ lora_offset,
+                              const int32_t *__restrict__ lora_rank, int n_adapters, int64_t R,
+                              int64_t t0, int nt, int tid, int nthr, int bar_id, DecodeTables &tb,
+                              int *off_out, int *rank_out) {
+  for (int k = tid; k < nt; k += nthr) tb.best[k] = ~0ull;
+  const bool staged = n_adapters <= kDecTable;
+  // the first pass of segments is loaded with the adapter tables, in one
+  // round; more segments than threads take further rounds
+  int32_t so0 = 0, so1 = 0, sa0 = 0;
+  if (tid < S) {
+    so0 = __ldg(seg_offsets + tid);
+    so1 = __ldg(seg_offsets + tid + 1);
+    sa0 = __ldg(seg_adapter + tid);
+  }
+  if (staged) {
+    for (int a = tid; a < n_adapters; a += nthr) {
+      tb.ad_off[a] = __ldg(lora_offset + a);
+      tb.ad_rank[a] = __ldg(lora_rank + a);
+    }
+  }
+  group_bar(bar_id, nthr);
+  for (int64_t s = tid; s < S; s += nthr) {
+    if (s != tid) {
+      so0 = __ldg(seg_offsets + s);
+      so1 = __ldg(seg_offsets + s + 1);
+      sa0 = __ldg(seg_adapter + s);
+    }
+    const int64_t lo = max(static_cast<int64_t>(so0), t0);
+    const int64_t hi = min(static_cast<int64_t>(so1), t0 + nt);
+    if (lo < hi) {
+      const unsigned long long key =
+          (static_cast<unsigned long long>(s) << 32) | static_cast<uint32_t>(sa0);
+      for (int64_t i = lo; i < hi; ++i) atomicMin(&tb.best[i - t0], key);
+    }
+  }
+  group_bar(bar_id, nthr);
+  for (int k = tid; k < nt; k += nthr) {
+    const unsigned long long key = tb.best[k];
+    int off = 0, r = 0;
+    if (key != ~0ull) {
+      const int a = static_cast<int>(static_cast<uint32_t>(key));
+      if (a < -1 || a >= n_adapters) {
+        record_device_error(SQ_ERR_BAD_SEGMENTS);
+      } else if (a >= 0) {
+        off = staged ? tb.ad_off[a] : __ldg(lora_offset + a);
+        r = staged ? tb.ad_rank[a] : __ldg(lora_rank + a);
+        if (off < 0 || (off & 15) || r <= 0 || r > kDecMaxRank || off + ((r + 15) & ~15) > R) {
+          record_device_error(SQ_ERR_BAD_SEGMENTS);
+          off = 0;
+          r = 0;
+        }
+      }
+    }
+    off_out[k] = off;
+    rank_out[k] = r;
+  }
+  group_bar(bar_id, nthr);
+}
+
+// ---------------------------------------------------------------------------
+// kernel 1: shrink partials.  Block (i, ks) writes
+//   part[(ks * M + i) * kDecMaxRank + j] = sum over its K slice of Xq[i,k] A'[off+j, k]
+// for j < r (no x_scale: the GEMM applies it to the sum of the slices).
+// Thread t covers 8 consecutive K elements per pass and loads the 16 A' rows
+// of a rank group together (all of the block's 16 x 4 KB at once).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kDecShrinkThreads, 2) decode_shrink_kernel(
+    const int8_t *__restrict__ Xq, int64_t M, int64_t K, int ksplit,
     const uint16_t *__restrict__ A_pack, const int32_t *__restrict__ lora_offset,
     const int32_t *__restrict__ lora_rank, int n_adapters, int64_t R,
     const int32_t *__restrict__ seg_offsets, const int32_t *__restrict__ seg_adapter, int64_t S,
@@ -43,93 +136,132 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_shrink_kernel(
   // nothing from here, and it waits for this grid to complete before it
   // reads the partial sums
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int unit = blockIdx.x * (kDecThreads / 32) + warp;  // (token, K slice)
-  const int64_t i = unit / kDecKSplit;
-  const int ks = unit % kDecKSplit;
-  if (i >= M) return;
-  int a = token_adapter(seg_offsets, seg_adapter, S, n_adapters, i);
-  int off = 0, r = 0;
-  if (a >= 0) {
-    off = lora_offset[a];
-    r = lora_rank[a];
-    if (off < 0 || (off & 15) || r <= 0 || r > kDecMaxRank || off + ((r + 15) & ~15) > R) {
-      if (lane == 0) record_device_error(SQ_ERR_BAD_SEGMENTS);
-      r = 0;
-    }
-  }
-  float *out = part + (i * kDecKSplit + ks) * kDecMaxRank;
-  // K slice of this warp, in 16-element pieces (K % 16 == 0); lane = piece
-  // (lane & 15) of each group of 16 pieces x half (lane >> 4) of each group
-  // of 16 ranks, so that all lanes load at once
-  const int64_t pieces = K / 16;
-  const int64_t p0 = pieces * ks / kDecKSplit, p1 = pieces * (ks + 1) / kDecKSplit;
-  const int pl = lane & 15, hf = lane >> 4;
-  // the codes and scales come from the quantizer (a no-op unless this grid
-  // is launched as its programmatic dependent)
+  __shared__ DecodeTables tb;
+  __shared__ int s_off, s_rank;
+  __shared__ float red[kDecShrinkThreads / 32][16];
+  const int64_t i = blockIdx.x / ksplit;
+  const int ks = static_cast<int>(blockIdx.x % ksplit);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  decode_lookup(seg_offsets, seg_adapter, S, lora_offset, lora_rank, n_adapters, R, i, 1, tid,
+                kDecShrinkThreads, 1, tb, &s_off, &s_rank);
+  const int off = s_off, r = s_rank;
+  if (r == 0) return;  // block-uniform
+  // the codes come from the quantizer (a no-op unless this grid is launched
+  // as its programmatic dependent)
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const float xs = x_scale[i];
+  const int64_t span = ((K + ksplit - 1) / ksplit + 7) / 8 * 8;
+  const int64_t k0 = ks * span, k1 = min(K, k0 + span);
+  const int8_t *xrow = Xq + i * K;
+  float *out = part + (static_cast<int64_t>(ks) * M + i) * kDecMaxRank;
   for (int j0 = 0; j0 < r; j0 += 16) {
-    const int jb = j0 + 8 * hf;  // this lane's 8 ranks (rows up to the padded rank exist)
-    float acc[8];
+    float acc[16];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-    for (int64_t p = p0 + pl; p < p1; p += 16) {
-      // all loads of this piece first, then the products
-      const uint4 xr = __ldg(reinterpret_cast<const uint4 *>(Xq + i * K + p * 16));
-      uint4 av[8][2];
+    for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+    for (int64_t k = k0 + 8 * tid; k < k1; k += 8 * kDecShrinkThreads) {
+      // rows off+j0 .. off+j0+15 exist (the pack pads every adapter to 16 rows)
+      const uint2 xv = __ldg(reinterpret_cast<const uint2 *>(xrow + k));
+      uint4 av[16];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint16_t *ap = A_pack + static_cast<int64_t>(off + jb + j) * K + p * 16;
-        av[j][0] = __ldg(reinterpret_cast<const uint4 *>(ap));
-        av[j][1] = __ldg(reinterpret_cast<const uint4 *>(ap + 8));
+      for (int j = 0; j < 16; ++j)
+        av[j] = __ldg(reinterpret_cast<const uint4 *>(A_pack + (off + j0 + j) * K + k));
+      float xf[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const uint32_t w = (t < 4) ? xv.x : xv.y;
+        xf[t] = static_cast<float>(static_cast<int8_t>((w >> (8 * (t & 3))) & 0xff));
       }
-      const uint32_t w4[4] = {xr.x, xr.y, xr.z, xr.w};
-      float xv[16];
 #pragma unroll
-      for (int t = 0; t < 16; ++t)
-        xv[t] = static_cast<float>(static_cast<int8_t>((w4[t >> 2] >> (8 * (t & 3))) & 0xff));
+      for (int j = 0; j < 16; ++j) {
+        const uint32_t a8[4] = {av[j].x, av[j].y, av[j].z, av[j].w};
+        float s = acc[j];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t a8[8] = {av[j][0].x, av[j][0].y, av[j][0].z, av[j][0].w,
-                                av[j][1].x, av[j][1].y, av[j][1].z, av[j][1].w};
-        float sacc = 0.f;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          sacc = fmaf(xv[2 * t], __uint_as_float(a8[t] << 16), sacc);
-          sacc = fmaf(xv[2 * t + 1], __uint_as_float(a8[t] & 0xffff0000u), sacc);
+        for (int t = 0; t < 4; ++t) {
+          s = fmaf(xf[2 * t], __uint_as_float(a8[t] << 16), s);
+          s = fmaf(xf[2 * t + 1], __uint_as_float(a8[t] & 0xffff0000u), s);
         }
-        acc[j] += sacc;
+        acc[j] = s;
       }
     }
-    // sum over the 16 piece lanes of each half, in a fixed order
+    // sum over the warp by halving exchanges (a fixed order): after the
+    // steps over lane bits 4..1 lane l holds rank (l >> 1) of the group
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float v = acc[j];
+    for (int o = 16, n = 8; o >= 2; o >>= 1, n >>= 1) {
+      const bool up = (lane & o) != 0;
 #pragma unroll
-      for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (pl == 0 && jb + j < r) out[jb + j] = xs * v;
+      for (int m = 0; m < n; ++m) {
+        const float send = up ? acc[m] : acc[m + n];
+        const float keep = up ? acc[m + n] : acc[m];
+        acc[m] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
     }
+    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
+    if ((lane & 1) == 0) red[warp][lane >> 1] = acc[0];
+    __syncthreads();
+    if (tid < 16 && j0 + tid < r) {
+      float t = 0.f;
+#pragma unroll
+      for (int w = 0; w < kDecShrinkThreads / 32; ++w) t += red[w][tid];
+      out[j0 + tid] = t;
+    }
+    __syncthreads();
   }
 }
 
+
 // ---------------------------------------------------------------------------
-// kernel 2: int8 GEMM over 32 output channels, then the LoRA expand.
-// Warp 8 streams this block's 32 rows of Wq and the tokens' Xq through a ring
-// of stages of 256 K-bytes, each two 128-byte-wide TMA tiles per operand
-// (128-byte swizzle: the 8 rows an MMA fragment load touches sit in distinct
-// banks); the four copies of a stage are issued by four lanes in one warp
-// instruction, since one thread's copies are issued one after another.
-// Compute warp w owns tokens [16*(w&3), +16) and channels [16*(w>>2), +16)
-// over the whole K, so no cross-warp reduction is needed.
+// kernel 2: int8 GEMM + LoRA expand on CTA pairs.
+// A tile is `tile_units` groups of 8 output channels (at most 64 channels);
+// tiles are dealt to the pairs in turn.  Per CTA and tile:
+//   warp 8 (producer) streams the CTA's K half in stages of two 128-byte K
+//     blocks: one TMA copy of the tile's Wq rows and one of the 64 Xq rows,
+//     each a 3D box over the K blocks (two boxes per operand per stage when
+//     K is not a multiple of 128), lanes 0 and 1 issuing together.  A copy
+//     costs a few hundred ns to issue whatever its size, so the copies are
+//     made large.  Before its first tile it also bulk-copies the B' rows of
+//     the CTA's output channels when the tokens use at least half of the
+//     pack's columns;
+//   warps 0-7 (compute): warp w owns tokens [16(w&3), +16) and channel groups
+//     [4(w>>2), +4) of the tile; the K loop's int32 partials go to shared
+//     memory, the pair adds them through distributed shared memory (CTA c
+//     keeps channels [c*half, (c+1)*half) of the tile), then the epilogue.
+// Loads that the tail depends on (peer partials, the shrink's partial sums,
+// w_scale) are all issued before any of them is used.  Every spin-wait is
+// bounded; all threads of both CTAs pass the same barriers in the same order,
+// also after a wait that ran out.
 // ---------------------------------------------------------------------------
-constexpr int kDecStages = 8;
-constexpr int kDecKStage = 256;                   // K bytes per stage (two tiles)
-constexpr int kDecWBytes = kDecCols * 128;        // Wq tile: 32 rows x 128 K-bytes
-constexpr int kDecXBytes = kDecMaxM * 128;        // Xq tile: 64 rows x 128 K-bytes
-constexpr int kDecStageBytes = 2 * (kDecWBytes + kDecXBytes);
+constexpr int kDecTileUnits = 8;                     // 8-channel groups per tile, at most
+constexpr int kDecRowsMax = 8 * kDecTileUnits;       // 64 output channels
+constexpr int kDecKbStage = 2;                       // 128-byte K blocks per stage
+constexpr int kDecStages = 4;
+constexpr int kDecWBytes = kDecKbStage * kDecRowsMax * 128;  // Wq slabs of a stage (16 KB)
+constexpr int kDecXBytes = kDecKbStage * kDecMaxM * 128;     // Xq slabs of a stage (16 KB)
+constexpr int kDecStageBytes = kDecWBytes + kDecXBytes;
+constexpr int kDecBBytes = (kDecRowsMax / 2) * SQ_MAX_LORA_COLS * 2;  // 64 KB
 constexpr int kDecComputeWarps = 8;
-constexpr int kDecGemmThreads = 32 * (kDecComputeWarps + 1);
+constexpr int kDecComputeThreads = 32 * kDecComputeWarps;
+constexpr int kDecGemmThreads = kDecComputeThreads + 32;
+// named barriers: 1 compute warps; 2 all warps after the token lookup;
+// 3 all warps after a tile's K loop; 4 all warps after a tile's epilogue
+constexpr int kBarCompute = 1, kBarLookup = 2, kBarRingFree = 3, kBarTileEnd = 4;
+
+struct DecodeCtl {
+  uint64_t full[kDecStages];
+  uint64_t empty[kDecStages];
+  uint64_t bfull;                  // B' rows landed
+  int tok_off[kDecMaxM];           // adapter column offset per token
+  int tok_rank[kDecMaxM];          // adapter rank per token (0: none)
+  float xs[kDecMaxM];              // x_scale per token
+  DecodeTables tb;
+  int abort;
+  int bdense;                      // B' rows staged in shared memory (first tile)
+};
+// after the K loop the ring holds the int32 partials [64][64] and then T [64][256] fp32
+constexpr int kDecPartBytes = kDecMaxM * kDecRowsMax * 4;
+static_assert(kDecPartBytes + kDecMaxM * kDecMaxRank * 4 <= kDecStages * kDecStageBytes,
+              "partials and T must fit the ring");
+
+constexpr size_t kDecSmemBytes =
+    static_cast<size_t>(kDecStages) * kDecStageBytes + kDecBBytes + sizeof(DecodeCtl) + 1024;
 
 __device__ __forceinline__ void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                              uint32_t b1) {
@@ -140,299 +272,399 @@ __device__ __forceinline__ void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4]
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-struct DecodeCtl {
-  uint64_t full[kDecStages];
-  uint64_t empty[kDecStages];
-  int off[kDecMaxM];               // adapter column offset per token
-  int rank[kDecMaxM];              // adapter rank per token (0: none)
-  int abort;
-};
-// the LoRA intermediate T[kDecMaxM][kDecMaxRank] (fp32) reuses the ring once
-// the K loop is over
-static_assert(kDecStages * kDecStageBytes >= kDecMaxM * kDecMaxRank * 4, "T must fit the ring");
-static_assert(32 * 8 == 4 * kDecMaxM, "four T threads per token");
+// 8 bf16 (one 16-byte word) times 8 fp32 values, added to d
+__device__ __forceinline__ float dot8_bf16(const uint4 &w, const float4 &t0, const float4 &t1,
+                                           float d) {
+  d = fmaf(t0.x, __uint_as_float(w.x << 16), d);
+  d = fmaf(t0.y, __uint_as_float(w.x & 0xffff0000u), d);
+  d = fmaf(t0.z, __uint_as_float(w.y << 16), d);
+  d = fmaf(t0.w, __uint_as_float(w.y & 0xffff0000u), d);
+  d = fmaf(t1.x, __uint_as_float(w.z << 16), d);
+  d = fmaf(t1.y, __uint_as_float(w.z & 0xffff0000u), d);
+  d = fmaf(t1.z, __uint_as_float(w.w << 16), d);
+  d = fmaf(t1.w, __uint_as_float(w.w & 0xffff0000u), d);
+  return d;
+}
 
-constexpr size_t kDecSmemBytes = static_cast<size_t>(kDecStages) * kDecStageBytes + sizeof(DecodeCtl) + 1024;
-
-__global__ void __launch_bounds__(kDecGemmThreads) decode_gemm_kernel(
+// (at most 112 registers a thread: a block of the shrink fits beside it on an SM)
+__global__ void __launch_bounds__(kDecGemmThreads, 2) decode_gemm_kernel(
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-    const float *__restrict__ x_scale, const float *__restrict__ w_scale, int64_t M, int64_t N,
-    int64_t K, int mode, const uint16_t *__restrict__ B_pack,
+    int view3d, const float *__restrict__ x_scale, const float *__restrict__ w_scale, int64_t M,
+    int64_t N, int64_t K, int mode, const uint16_t *__restrict__ B_pack,
     const int32_t *__restrict__ lora_offset, const int32_t *__restrict__ lora_rank,
     int n_adapters, int64_t R, const int32_t *__restrict__ seg_offsets,
-    const int32_t *__restrict__ seg_adapter, int64_t S, const float *__restrict__ part,
-    void *__restrict__ out, uint64_t timeout_ns) {
+    const int32_t *__restrict__ seg_adapter, int64_t S, const float *part, int ksplit,
+    int tile_units, int tiles, void *__restrict__ out, uint64_t timeout_ns) {
   extern __shared__ uint8_t dsm_raw[];
   uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
-  DecodeCtl &ctl = *reinterpret_cast<DecodeCtl *>(ring + kDecStages * kDecStageBytes);
+  uint16_t *bsm = reinterpret_cast<uint16_t *>(ring + kDecStages * kDecStageBytes);
+  DecodeCtl &ctl = *reinterpret_cast<DecodeCtl *>(ring + kDecStages * kDecStageBytes + kDecBBytes);
+  int *P = reinterpret_cast<int *>(ring);                          // [64][64] int32
+  float *Tm = reinterpret_cast<float *>(ring + kDecPartBytes);     // [64][256] fp32
   volatile int *abort_flag = &ctl.abort;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kDecCols;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t crank = cluster_ctarank();
+  const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
   const bool lora = (part != nullptr);
-  const int nk = (mode == 2) ? 0 : static_cast<int>((K + kDecKStage - 1) / kDecKStage);
-  const int kb_first = (nk > 0) ? static_cast<int>((blockIdx.x * 5u) % static_cast<unsigned>(nk)) : 0;
+  const int tile_rows = 8 * tile_units, half = 4 * tile_units;
+  const int slab_w = tile_rows * 128;  // bytes of one K block of the Wq tile
+  const int nk = (mode == 2) ? 0 : static_cast<int>((K + 127) / 128);
+  const int nk_half = (nk + 1) / 2;
+  const int kb0 = static_cast<int>(crank) * nk_half;
+  const int my_nk = max(0, min(nk, kb0 + nk_half) - kb0);
+  const int nstage = (my_nk + kDecKbStage - 1) / kDecKbStage;
+  const int mt = static_cast<int>(min(M, static_cast<int64_t>(kDecMaxM)));
 
   if (threadIdx.x == 0) {
-    for (int st = 0; st < kDecStages; ++st) {
-      mbar_init(&ctl.full[st], 1);
-      mbar_init(&ctl.empty[st], kDecComputeWarps);
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(&ctl.full[s], 1);
+      mbar_init(&ctl.empty[s], kDecComputeWarps);
     }
+    mbar_init(&ctl.bfull, 1);
     ctl.abort = 0;
+    ctl.bdense = 0;
     fence_mbar_init();
   }
   __syncthreads();
 
   if (warp == kDecComputeWarps) {
     // ---------------------------------------------------------- producer
-    // lane 0 waits for a free stage and posts its bytes; lanes 0-3 then copy
-    // Wq tile 0, Wq tile 1, Xq tile 0 and Xq tile 1 of the stage together
-    int issued = 0;
-    {
-      if (lane == 0) {
-        prefetch_tmap(&tm_w);
-        prefetch_tmap(&tm_x);
-      }
-      uint32_t phase = 0;
-      int st = 0;
-      // blocks start their K walk at different stages so that they do not
-      // all read the same Xq tile (from the same L2 lines) at once
-      int kk = kb_first;
-      for (int kb = 0; kb < nk; ++kb) {
-        bool got = true;
-        if (lane == 0) {
-          got = mbar_wait(&ctl.empty[st], phase ^ 1u, timeout_ns, abort_flag);
-          if (got) mbar_arrive_expect_tx(&ctl.full[st], kDecStageBytes);
+    if (lane == 0) {
+      prefetch_tmap(&tm_w);
+      prefetch_tmap(&tm_x);
+    }
+    int q = 0;  // stages issued so far (all tiles)
+    bool looked_up = false, b_issued = false, stop = false;
+    auto after_lookup = [&](int first_tile) {
+      // B' rows of this CTA's channels in the first tile, when the tokens use
+      // at least half of the pack's columns (else the epilogue reads the used
+      // columns from global memory)
+      group_bar(kBarLookup, kDecGemmThreads);
+      looked_up = true;
+      if (!lora || first_tile >= tiles || lane != 0 || R <= 0) return;
+      unsigned long long used = 0;  // 16-column groups (R <= 1024)
+      for (int i = 0; i < mt; ++i) {
+        const int r = ctl.tok_rank[i];
+        if (r > 0) {
+          const int g0 = ctl.tok_off[i] >> 4, g1 = (ctl.tok_off[i] + r + 15) >> 4;
+          for (int g = g0; g < g1; ++g) used |= 1ull << g;
         }
-        if (!__shfl_sync(0xffffffffu, got, 0)) {
-          if (lane == 0) {
+      }
+      if (2 * 16 * __popcll(used) < R) return;
+      const int64_t c0 = static_cast<int64_t>(first_tile) * tile_rows + crank * half;
+      const int64_t rows = max(static_cast<int64_t>(0), min(static_cast<int64_t>(half), N - c0));
+      if (rows <= 0) return;
+      const uint32_t bytes = static_cast<uint32_t>(rows * R * 2);
+      ctl.bdense = 1;
+      mbar_arrive_expect_tx(&ctl.bfull, bytes);
+      bulk_load(bsm, B_pack + c0 * R, bytes, &ctl.bfull);
+      b_issued = true;
+    };
+    for (int tile = pair; tile < tiles; tile += npairs) {
+      const int32_t n0 = tile * tile_rows;
+      for (int si = 0; si < nstage; ++si) {
+        const int slot = q % kDecStages;
+        const uint32_t ph = static_cast<uint32_t>(q / kDecStages) & 1u;
+        const int kbs = kb0 + si * kDecKbStage;                       // first K block
+        const int nkb = min(kDecKbStage, kb0 + my_nk - kbs);          // this CTA's blocks
+        const int boxes = view3d ? kDecKbStage : nkb;                 // K blocks copied
+        bool got = true;
+        if (lane == 0 && !stop) {
+          // nothing more is issued once any wait has run out: a slot whose
+          // copy nobody waited for may still be written to
+          got = !*abort_flag && mbar_wait(&ctl.empty[slot], ph ^ 1u, timeout_ns, abort_flag) &&
+                !*abort_flag;
+          if (got)
+            mbar_arrive_expect_tx(&ctl.full[slot],
+                                  static_cast<uint32_t>(boxes * (slab_w + kDecMaxM * 128)));
+        }
+        got = __shfl_sync(0xffffffffu, got && !stop, 0);
+        if (!got) {
+          if (lane == 0 && !stop) {
             *reinterpret_cast<volatile int *>(abort_flag) = 1;
             record_device_error(SQ_ERR_DEVICE_TIMEOUT);
           }
-          break;
+          stop = true;
+        } else {
+          uint8_t *st = ring + slot * kDecStageBytes;
+          if (view3d) {
+            if (lane == 0) tma_load_3d(st, &tm_w, &ctl.full[slot], 0, n0, kbs);
+            if (lane == 1) tma_load_3d(st + kDecWBytes, &tm_x, &ctl.full[slot], 0, 0, kbs);
+          } else if (lane < 2 * nkb) {
+            const int kb = lane >> 1;
+            if ((lane & 1) == 0)
+              tma_load_2d(st + kb * slab_w, &tm_w, &ctl.full[slot], (kbs + kb) * 128, n0);
+            else
+              tma_load_2d(st + kDecWBytes + kb * kDecMaxM * 128, &tm_x, &ctl.full[slot],
+                          (kbs + kb) * 128, 0);
+          }
+          ++q;
         }
-        if (lane < 4) {
-          const int tile = lane & 1;  // K half of the stage
-          const int32_t x = kk * kDecKStage + tile * 128;
-          if (lane < 2)
-            tma_load_2d(ring + st * kDecStageBytes + tile * kDecWBytes, &tm_w, &ctl.full[st], x,
-                        static_cast<int32_t>(n0));
-          else
-            tma_load_2d(ring + st * kDecStageBytes + 2 * kDecWBytes + tile * kDecXBytes, &tm_x,
-                        &ctl.full[st], x, 0);
-        }
-        ++issued;
-        if (++kk == nk) kk = 0;
-        if (++st == kDecStages) { st = 0; phase ^= 1u; }
+        if (!looked_up && (q == kDecStages || si == nstage - 1)) after_lookup(pair);
       }
-    }
-    if (lane == 0) {
-      // every issued copy must land before the block exits: wait for the
-      // last use of each stage
-      volatile int never = 0;
-      for (int s2 = 0; s2 < kDecStages && s2 < issued; ++s2) {
-        const int last_kb = issued - 1 - ((issued - 1 - s2) % kDecStages);
-        const uint32_t par = static_cast<uint32_t>((last_kb / kDecStages) & 1);
-        mbar_wait(&ctl.full[s2], par, 1000000000ull, &never);
-      }
-    }
-  } else {
-    // --------------------------------------------------------- compute
-    const int mt = warp & 3, nh = warp >> 2;
-    int acc[2][4];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[nt][e] = 0;
-    const int ra = mt * 16 + g, rb = ra + 8;  // token rows of this lane's A fragments
-    // adapter of each token (warps 0-3 cover the 64 tokens), looked up while
-    // the first stages load; read by all compute warps after the K loop
-    if (lora && nh == 0 && lane < 16) {
-      const int i = mt * 16 + lane;
-      int off = 0, r = 0;
-      if (i < M) {
-        const int a = token_adapter(seg_offsets, seg_adapter, S, n_adapters, i);
-        if (a >= 0) {
-          off = lora_offset[a];
-          r = lora_rank[a];
-          if (off < 0 || (off & 15) || r <= 0 || r > kDecMaxRank || off + ((r + 15) & ~15) > R)
-            r = 0;
+      if (!looked_up) after_lookup(pair);
+      // every copy of this tile must land before the ring is reused (also
+      // after a wait that ran out: wait for the last use of each slot)
+      if (lane == 0) {
+        volatile int never = 0;
+        const int issued = q;
+        for (int k = 0; k < kDecStages && k < issued; ++k) {
+          const int last = issued - 1 - ((issued - 1 - k) % kDecStages);
+          mbar_wait(&ctl.full[last % kDecStages], static_cast<uint32_t>(last / kDecStages) & 1u,
+                    1000000000ull, &never);
         }
-      }
-      ctl.off[i] = off;
-      ctl.rank[i] = r;
-    }
-    uint32_t phase = 0;
-    int st = 0;
-    bool ok = true;
-    for (int kb = 0; kb < nk; ++kb) {
-      // the warp leaves together: the mma.sync below needs all lanes
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ctl.full[st], phase, timeout_ns, abort_flag))))
-        break;
-#pragma unroll
-      for (int hh = 0; hh < 4; ++hh) {
-        const int h = hh & 1;  // 64-byte half of a 128-byte tile row
-        const uint8_t *wt = ring + st * kDecStageBytes + (hh >> 1) * kDecWBytes;
-        const uint8_t *xt = ring + st * kDecStageBytes + 2 * kDecWBytes + (hh >> 1) * kDecXBytes;
-        // 16 contiguous K bytes (chunk 4h + tig of the 128-byte row, stored
-        // 128B-swizzled) of each operand row; the K order inside the 64 bytes
-        // is a permutation that A and B share
-        const uint4 xa = *reinterpret_cast<const uint4 *>(xt + ra * 128 + (((4 * h + tig) ^ (ra & 7)) * 16));
-        const uint4 xb = *reinterpret_cast<const uint4 *>(xt + rb * 128 + (((4 * h + tig) ^ (rb & 7)) * 16));
-        const uint32_t fa0[4] = {xa.x, xb.x, xa.y, xb.y};
-        const uint32_t fa1[4] = {xa.z, xb.z, xa.w, xb.w};
-        uint4 bw[2];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          const int row = nh * 16 + nt * 8 + g;
-          bw[nt] = *reinterpret_cast<const uint4 *>(wt + row * 128 + (((4 * h + tig) ^ (row & 7)) * 16));
-        }
-        // independent accumulators back to back
-        mma_s8_16832(acc[0], fa0, bw[0].x, bw[0].y);
-        mma_s8_16832(acc[1], fa0, bw[1].x, bw[1].y);
-        mma_s8_16832(acc[0], fa1, bw[0].z, bw[0].w);
-        mma_s8_16832(acc[1], fa1, bw[1].z, bw[1].w);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl.empty[st]);
-      if (++st == kDecStages) { st = 0; phase ^= 1u; }
+      group_bar(kBarRingFree, kDecGemmThreads);
+      cluster_sync();  // partials written by both CTAs
+      cluster_sync();  // partials read by both CTAs
+      group_bar(kBarTileEnd, kDecGemmThreads);
+    }
+    if (!looked_up) after_lookup(pair);
+    if (lane == 0 && b_issued) {
+      volatile int never = 0;
+      mbar_wait(&ctl.bfull, 0, 1000000000ull, &never);
+    }
+    return;
+  }
+
+  // ----------------------------------------------------------- compute
+  const int tid = threadIdx.x;
+  const int g = lane >> 2, tig = lane & 3;
+  if (lora)
+    decode_lookup(seg_offsets, seg_adapter, S, lora_offset, lora_rank, n_adapters, R, 0, mt, tid,
+                  kDecComputeThreads, kBarCompute, ctl.tb, ctl.tok_off, ctl.tok_rank);
+  else
+    for (int i = tid; i < kDecMaxM; i += kDecComputeThreads) ctl.tok_rank[i] = 0;
+  for (int i = tid; i < kDecMaxM; i += kDecComputeThreads)
+    ctl.xs[i] = (mode != 1 && i < M) ? __ldg(x_scale + i) : 0.f;
+  group_bar(kBarLookup, kDecGemmThreads);
+
+  const int mtile = warp & 3, ng = warp >> 2;
+  const int ra = mtile * 16 + g, rb = ra + 8;  // token rows of this lane's A fragments
+  int q = 0;
+  bool first = true;
+  for (int tile = pair; tile < tiles; tile += npairs) {
+    const int64_t n0 = static_cast<int64_t>(tile) * tile_rows;
+    const int64_t c0 = n0 + static_cast<int64_t>(crank) * half;  // this CTA's first channel
+    const int tok = tid >> 2;                                       // epilogue token
+    const int npairs_out = half / 2;
+    // w_scale of this thread's epilogue channels, loaded ahead of every wait
+    float wsv[4][2];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int p = (tid & 3) + 4 * m;
+      const int64_t n = c0 + 2 * p;
+      const bool ok_n = mode == 0 && p < npairs_out && n < N;
+      wsv[m][0] = ok_n ? __ldg(w_scale + n) : 0.f;
+      wsv[m][1] = ok_n ? __ldg(w_scale + n + 1) : 0.f;
+    }
+    int acc[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[u][e] = 0;
+    bool ok = true;
+    for (int si = 0; si < nstage; ++si, ++q) {
+      const int slot = q % kDecStages;
+      const uint32_t ph = static_cast<uint32_t>(q / kDecStages) & 1u;
+      // the warp leaves together: the mma.sync below needs all lanes.  A warp
+      // whose wait ran out raises the abort flag at once and hands no more
+      // stages back (the producer then issues nothing more)
+      if (ok) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&ctl.full[slot], ph, timeout_ns, abort_flag));
+        if (!ok && lane == 0) *reinterpret_cast<volatile int *>(abort_flag) = 1;
+      }
+      if (!ok) continue;
+      const int nkb = min(kDecKbStage, my_nk - si * kDecKbStage);
+      for (int kb = 0; kb < nkb; ++kb) {
+        const uint8_t *wt = ring + slot * kDecStageBytes + kb * slab_w;
+        const uint8_t *xt = ring + slot * kDecStageBytes + kDecWBytes + kb * kDecMaxM * 128;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          // 16 contiguous K bytes (chunk 4h + tig of the 128-byte row, stored
+          // 128B-swizzled) of each operand row; the K order inside the 64
+          // bytes is a permutation that A and B share
+          const uint4 xa = *reinterpret_cast<const uint4 *>(xt + ra * 128 + (((4 * h + tig) ^ (ra & 7)) * 16));
+          const uint4 xb = *reinterpret_cast<const uint4 *>(xt + rb * 128 + (((4 * h + tig) ^ (rb & 7)) * 16));
+          const uint32_t fa0[4] = {xa.x, xb.x, xa.y, xb.y};
+          const uint32_t fa1[4] = {xa.z, xb.z, xa.w, xb.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (ng * 4 + u >= tile_units) continue;  // warp-uniform
+            const int row = (ng * 4 + u) * 8 + g;
+            const uint4 bw = *reinterpret_cast<const uint4 *>(wt + row * 128 + (((4 * h + tig) ^ (row & 7)) * 16));
+            mma_s8_16832(acc[u], fa0, bw.x, bw.y);
+            mma_s8_16832(acc[u], fa1, bw.z, bw.w);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl.empty[slot]);
     }
     if (!ok) {
       *reinterpret_cast<volatile int *>(abort_flag) = 1;
       record_device_error(SQ_ERR_DEVICE_TIMEOUT);
     }
-    // ---- LoRA: every compute warp has finished reading the ring (T may
-    //      overwrite it) and the adapter table is complete; the B' columns of
-    //      the first 16 ranks are loaded before the shrink's partial sums are
-    //      waited for, then T = sum of the partials over the shrink's K slices.
-    //      Every compute warp meets both barriers, also after a wait that ran out.
-    float (*Tm)[kDecMaxRank] = reinterpret_cast<float (*)[kDecMaxRank]>(ring);
-    asm volatile("bar.sync 1, %0;" ::"r"(32 * kDecComputeWarps) : "memory");
-    // lane: rows ra, rb; channels n0 + 16nh + 8nt + 2tig + {0,1}
-    float d[2][2][2];  // [half][nt][channel of the pair]
-    int rr[2], oo[2];
+    // every copy into the ring has landed (the producer waited): the
+    // partials go where the stages were
+    group_bar(kBarRingFree, kDecGemmThreads);
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int i = half ? rb : ra;
-      rr[half] = (lora && i < M) ? ctl.rank[i] : 0;
-      oo[half] = (lora && i < M) ? ctl.off[i] : 0;
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) d[half][nt][0] = d[half][nt][1] = 0.f;
+    for (int u = 0; u < 4; ++u) {
+      const int c = (ng * 4 + u) * 8 + 2 * tig;
+      *reinterpret_cast<int2 *>(P + ra * kDecRowsMax + c) = make_int2(acc[u][0], acc[u][1]);
+      *reinterpret_cast<int2 *>(P + rb * kDecRowsMax + c) = make_int2(acc[u][2], acc[u][3]);
     }
-    const int rmax = max(rr[0], rr[1]);
-    auto load_b = [&](int j0, uint4 (&bv)[2][2][2]) {
+    cluster_sync();
+    // this CTA keeps channels [crank*half, (crank+1)*half) of the tile: token
+    // tok = tid/4, channel pairs p = tid%4 + 4m; its own partial plus the
+    // peer's, every load issued before the first add
+    const uint32_t peer = crank ^ 1u;
+    int2 own[4], oth[4];
 #pragma unroll
-      for (int half = 0; half < 2; ++half)
+    for (int m = 0; m < 4; ++m) {
+      const int p = (tid & 3) + 4 * m;
+      own[m] = make_int2(0, 0);
+      oth[m] = make_int2(0, 0);
+      if (p < npairs_out) {
+        const int c = static_cast<int>(crank) * half + 2 * p;
+        own[m] = *reinterpret_cast<const int2 *>(P + tok * kDecRowsMax + c);
+        oth[m] = ld_cluster_i2(map_to_rank(smem_u32(P + tok * kDecRowsMax + c), peer));
+      }
+    }
+    int2 accv[4];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          const int64_t n = n0 + nh * 16 + nt * 8 + 2 * tig;
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-            bv[half][nt][c] = (j0 < rr[half] && n + c < N)
-                                  ? __ldg(reinterpret_cast<const uint4 *>(B_pack + (n + c) * R + oo[half] + j0))
-                                  : make_uint4(0, 0, 0, 0);
-        }
-    };
-    uint4 bpre[2][2][2][2];  // column groups 0 and 1 (ranks 0-15), loaded early
-    load_b(0, bpre[0]);
-    load_b(8, bpre[1]);
-    if (lora) {
+    for (int m = 0; m < 4; ++m) accv[m] = make_int2(own[m].x + oth[m].x, own[m].y + oth[m].y);
+    cluster_sync();
+    // ---- LoRA: T = x_scale * (sum of the shrink's slices in order), after
+    //      the shrink grid has completed; each thread takes four (token, rank)
+    //      entries of a 16-rank group and loads all their slices at once
+    const int r_i = (tok < mt) ? ctl.tok_rank[tok] : 0;
+    const int off_i = (tok < mt) ? ctl.tok_off[tok] : 0;
+    const bool any_lora = lora && mode != 1;
+    if (any_lora) {
       asm volatile("griddepcontrol.wait;" ::: "memory");
-      // four threads per token, each summing every fourth column; the 16
-      // partials of four columns are loaded before any is added
-      const int i = threadIdx.x >> 2, jq = threadIdx.x & 3;
-      const int r = (i < M) ? ctl.rank[i] : 0;
-      const int rpad = (r + 15) & ~15;
-      for (int jb = 0; jb < rpad; jb += 16) {
-        float pv[4][kDecKSplit];
+      int rmax = 0;
+      for (int t = 0; t < mt; ++t) rmax = max(rmax, ctl.tok_rank[t]);
+      for (int jb = 0; jb < rmax; jb += 16) {
+        const int j = jb + (tid & 15);
+        float pv[4][kDecShrinkSplitMax];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int j = jb + jq + 4 * m;
+        for (int u = 0; u < 4; ++u) {
+          const int t = (tid >> 4) + 16 * u;
+          const int r = (t < mt) ? ctl.tok_rank[t] : 0;
 #pragma unroll
-          for (int ks = 0; ks < kDecKSplit; ++ks)
-            pv[m][ks] = (j < r) ? part[(i * kDecKSplit + ks) * kDecMaxRank + j] : 0.f;
+          for (int ks = 0; ks < kDecShrinkSplitMax; ++ks)
+            pv[u][ks] = (j < r && ks < ksplit)
+                            ? part[(static_cast<int64_t>(ks) * M + t) * kDecMaxRank + j]
+                            : 0.f;
         }
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          float t = 0.f;  // zero in the padding columns (the expand reads them)
+        for (int u = 0; u < 4; ++u) {
+          const int t = (tid >> 4) + 16 * u;
+          const int r = (t < mt) ? ctl.tok_rank[t] : 0;
+          if (t < mt && j < ((r + 15) & ~15)) {
+            float sacc = 0.f;  // zero in the padding columns
 #pragma unroll
-          for (int ks = 0; ks < kDecKSplit; ++ks) t += pv[m][ks];
-          Tm[i][jb + jq + 4 * m] = t;
-        }
-      }
-      asm volatile("bar.sync 1, %0;" ::"r"(32 * kDecComputeWarps) : "memory");
-    }
-    for (int j0 = 0; j0 < rmax; j0 += 8) {
-      uint4 bv[2][2][2];  // [half][nt][channel]
-      if (j0 == 0) {
-#pragma unroll
-        for (int half = 0; half < 2; ++half)
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int c = 0; c < 2; ++c) bv[half][nt][c] = bpre[0][half][nt][c];
-      } else if (j0 == 8) {
-#pragma unroll
-        for (int half = 0; half < 2; ++half)
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int c = 0; c < 2; ++c) bv[half][nt][c] = bpre[1][half][nt][c];
-      } else {
-        load_b(j0, bv);
-      }
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        if (j0 >= rr[half]) continue;
-        const int i = half ? rb : ra;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const uint32_t w[4] = {bv[half][nt][c].x, bv[half][nt][c].y, bv[half][nt][c].z,
-                                   bv[half][nt][c].w};
-            float acc_d = d[half][nt][c];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              acc_d = fmaf(Tm[i][j0 + 2 * t], __uint_as_float(w[t] << 16), acc_d);
-              acc_d = fmaf(Tm[i][j0 + 2 * t + 1], __uint_as_float(w[t] & 0xffff0000u), acc_d);
-            }
-            d[half][nt][c] = acc_d;
+            for (int ks = 0; ks < kDecShrinkSplitMax; ++ks) sacc += pv[u][ks];
+            Tm[t * kDecMaxRank + j] = __fmul_rn(ctl.xs[t], sacc);
           }
-      }
-    }
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int64_t i = half ? rb : ra;
-      if (i >= M) continue;
-      const float xs = (mode == 0) ? x_scale[i] : 0.f;
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int64_t n = n0 + nh * 16 + nt * 8 + 2 * tig;
-        if (n >= N) continue;  // N % 16 == 0: both channels of the pair exist
-        const int s0 = acc[nt][2 * half], s1 = acc[nt][2 * half + 1];
-        const float d0 = d[half][nt][0], d1 = d[half][nt][1];
-        if (mode == 0) {
-          const float y0 = __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(s0), xs), __ldg(w_scale + n)), d0);
-          const float y1 = __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(s1), xs), __ldg(w_scale + n + 1)), d1);
-          __nv_bfloat162 hh = __floats2bfloat162_rn(y0, y1);
-          *reinterpret_cast<uint32_t *>(static_cast<uint16_t *>(out) + i * N + n) =
-              *reinterpret_cast<uint32_t *>(&hh);
-        } else if (mode == 1) {
-          *reinterpret_cast<int2 *>(static_cast<int32_t *>(out) + i * N + n) = make_int2(s0, s1);
-        } else {
-          *reinterpret_cast<float2 *>(static_cast<float *>(out) + i * N + n) = make_float2(d0, d1);
         }
       }
+      group_bar(kBarCompute, kDecComputeThreads);
     }
+    const bool use_bsm = first && ctl.bdense;
+    if (use_bsm && !mbar_wait(&ctl.bfull, 0, timeout_ns, abort_flag)) {
+      *reinterpret_cast<volatile int *>(abort_flag) = 1;
+      record_device_error(SQ_ERR_DEVICE_TIMEOUT);
+    }
+    const bool aborted = *abort_flag != 0;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int p = (tid & 3) + 4 * m;
+      const int64_t n = c0 + 2 * p;
+      if (p >= npairs_out || tok >= mt || n >= N || aborted) continue;
+      float d0 = 0.f, d1 = 0.f;
+      if (any_lora && r_i > 0) {
+        const float *Ti = Tm + tok * kDecMaxRank;
+        for (int j = 0; j < r_i; j += 8) {
+          const float4 t0 = *reinterpret_cast<const float4 *>(Ti + j);
+          const float4 t1 = *reinterpret_cast<const float4 *>(Ti + j + 4);
+          uint4 w0, w1;
+          if (use_bsm) {
+            w0 = *reinterpret_cast<const uint4 *>(bsm + (n - c0) * R + off_i + j);
+            w1 = *reinterpret_cast<const uint4 *>(bsm + (n + 1 - c0) * R + off_i + j);
+          } else {
+            w0 = __ldg(reinterpret_cast<const uint4 *>(B_pack + n * R + off_i + j));
+            w1 = __ldg(reinterpret_cast<const uint4 *>(B_pack + (n + 1) * R + off_i + j));
+          }
+          d0 = dot8_bf16(w0, t0, t1, d0);
+          d1 = dot8_bf16(w1, t0, t1, d1);
+        }
+      }
+      if (mode == 0) {
+        const float xs = ctl.xs[tok];
+        const float y0 = __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(accv[m].x), xs), wsv[m][0]), d0);
+        const float y1 = __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(accv[m].y), xs), wsv[m][1]), d1);
+        __nv_bfloat162 hh = __floats2bfloat162_rn(y0, y1);
+        *reinterpret_cast<uint32_t *>(static_cast<uint16_t *>(out) + tok * N + n) =
+            *reinterpret_cast<uint32_t *>(&hh);
+      } else if (mode == 1) {
+        *reinterpret_cast<int2 *>(static_cast<int32_t *>(out) + tok * N + n) = accv[m];
+      } else {
+        *reinterpret_cast<float2 *>(static_cast<float *>(out) + tok * N + n) = make_float2(d0, d1);
+      }
+    }
+    first = false;
+    group_bar(kBarTileEnd, kDecGemmThreads);
   }
 }
 
 size_t decode_workspace_bytes(int64_t M) {
-  return static_cast<size_t>(M) * kDecKSplit * kDecMaxRank * sizeof(float);
+  return static_cast<size_t>(kDecShrinkSplitMax) * static_cast<size_t>(M) * kDecMaxRank *
+         sizeof(float);
 }
 
 bool decode_applicable(int64_t M) { return M > 0 && M <= kDecMaxM; }
+
+// CTA pairs of decode_gemm_kernel that fit on the current device at once
+// (cached per device).  On first use per device the kernels' shared-memory
+// settings are made: the GEMM's opt-in, and the shrink's preference for the
+// largest shared-memory carveout, so that an SM running shrink blocks keeps
+// room for a GEMM CTA beside them (a block pins its SM's carveout, and an SM
+// split for a small-shared-memory kernel cannot host the GEMM until it empties).
+static cudaError_t decode_pairs(int *pairs) {
+  static std::atomic<int> attr_set[kMaxDevices];
+  static std::atomic<int> cached[kMaxDevices];
+  const int dev = current_device_index();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
+    cudaError_t e = ensure_smem_optin(decode_gemm_kernel, static_cast<int>(kDecSmemBytes), attr_set);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(decode_shrink_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(kDecGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = kDecSmemBytes;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    e = cudaOccupancyMaxActiveClusters(&n, decode_gemm_kernel, &cfg);
+    if (e != cudaSuccess) return e;
+    n = n > 0 ? n : sm_count_of_current_device() / 2;
+    cached[dev].store(n, std::memory_order_relaxed);
+  }
+  *pairs = n;
+  return cudaSuccess;
+}
 
 // mode: 0 = Y bf16, 1 = int32 accumulators, 2 = LoRA delta fp32.
 // `part` (scratch, decode_workspace_bytes(M)) may be null when there is no LoRA.
@@ -443,44 +675,57 @@ cudaError_t launch_decode(const int8_t *Xq, const float *x_scale, const int8_t *
                           int64_t R, const int32_t *seg_offsets, const int32_t *seg_adapter,
                           int64_t S, float *part, void *out, cudaStream_t st) {
   const bool lora = part != nullptr && mode != 1;
+  int max_pairs = 0;
+  cudaError_t e = decode_pairs(&max_pairs);
+  if (e != cudaSuccess) return e;
+  int ksplit = static_cast<int>((K + kDecShrinkSpan - 1) / kDecShrinkSpan);
+  ksplit = ksplit < 1 ? 1 : (ksplit > kDecShrinkSplitMax ? kDecShrinkSplitMax : ksplit);
   if (lora) {
-    const int units = static_cast<int>(M) * kDecKSplit;
-    const int blocks = (units + kDecThreads / 32 - 1) / (kDecThreads / 32);
-    decode_shrink_kernel<<<blocks, kDecThreads, 0, st>>>(Xq, x_scale, M, K, A_pack, lora_offset,
-                                                         lora_rank, n_adapters, R, seg_offsets,
-                                                         seg_adapter, S, part);
-    cudaError_t e = cudaGetLastError();
+    decode_shrink_kernel<<<static_cast<unsigned>(M * ksplit), kDecShrinkThreads, 0, st>>>(
+        Xq, M, K, ksplit, A_pack, lora_offset, lora_rank, n_adapters, R, seg_offsets, seg_adapter,
+        S, part);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
+  // tiles of up to 8 groups of 8 channels, sized so that the pairs that fit
+  // on the device get one tile each where N allows
+  const int64_t units = N / 8;
+  const int64_t per = (units + max_pairs - 1) / max_pairs;
+  const int tile_units = static_cast<int>(per < 1 ? 1 : (per > kDecTileUnits ? kDecTileUnits : per));
+  const int64_t tiles = (units + tile_units - 1) / tile_units;
+  const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
   CUtensorMap tm_w, tm_x;
   memset(&tm_w, 0, sizeof tm_w);
   memset(&tm_x, 0, sizeof tm_x);
-  if (mode != 2 &&
-      (!make_tmap(&tm_w, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, 128, kDecCols) ||
-       !make_tmap(&tm_x, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, 128, kDecMaxM)))
-    return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(decode_gemm_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kDecSmemBytes));
-    if (e != cudaSuccess) return e;
-    attr = true;
+  // K a multiple of 128: one 3D box per operand and stage; otherwise one 2D
+  // box per K block (the last block's tail is filled with zeros)
+  const int view3d = (K % 128 == 0) ? 1 : 0;
+  if (mode != 2) {
+    const bool made =
+        view3d ? (make_tmap_kblocks(&tm_w, Wq, K, N, 8 * tile_units, kDecKbStage) &&
+                  make_tmap_kblocks(&tm_x, Xq, K, M, kDecMaxM, kDecKbStage))
+               : (make_tmap(&tm_w, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, 128, 8 * tile_units) &&
+                  make_tmap(&tm_x, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, 128, kDecMaxM));
+    if (!made) return cudaErrorInvalidValue;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((N + kDecCols - 1) / kDecCols), 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
   cfg.blockDim = dim3(kDecGemmThreads, 1, 1);
   cfg.dynamicSmemBytes = kDecSmemBytes;
   cfg.stream = st;
-  cudaLaunchAttribute attrs[1];
-  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeClusterDimension;
+  attrs[0].val.clusterDim.x = 2;
+  attrs[0].val.clusterDim.y = 1;
+  attrs[0].val.clusterDim.z = 1;
+  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attrs;
-  cfg.numAttrs = lora ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, decode_gemm_kernel, tm_w, tm_x, x_scale, w_scale, M, N, K, mode,
-                            B_pack, lora_offset, lora_rank, n_adapters, R, seg_offsets,
-                            seg_adapter, S, lora ? static_cast<const float *>(part) : nullptr, out,
-                            wait_timeout_ns());
+  cfg.numAttrs = lora ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, decode_gemm_kernel, tm_w, tm_x, view3d, x_scale, w_scale, M, N,
+                            K, mode, B_pack, lora_offset, lora_rank, n_adapters, R, seg_offsets,
+                            seg_adapter, S, lora ? static_cast<const float *>(part) : nullptr,
+                            ksplit, tile_units, static_cast<int>(tiles), out, wait_timeout_ns());
 }
 
 }  // namespace sq

@@ -81,6 +81,8 @@ struct SharedCtl {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  uint32_t issued;           // stages this CTA's producer issued
+  uint32_t peer_issued;      // first CTA: stages the second CTA's producer issued
 };
 
 static_assert(sizeof(SharedCtl) <= 1024, "control block fits its 1 KB slot");
@@ -224,6 +226,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
+    ctl->issued = 0;
+    ctl->peer_issued = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -273,6 +277,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tma_load_2d_pair(a_dst + kABytes, &tm_bp, full_pair, a * kLoraChunk, nb * BN + row_off);
         }
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        ++ctl->issued;
         return true;
       });
       if (!ok) signal_abort(ctl);
@@ -454,13 +459,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0) bulk_wait_group<0>();  // this warp's output stores are complete
   }
 
-  if (*abort_flag) {
-    // a stopped pair may still have copies in flight: give them time to land
-    const uint64_t t0 = globaltimer_ns();
-    while (globaltimer_ns() - t0 < 100000ull) {
+  // Copies of both CTAs complete on the first CTA's `full` barriers, which
+  // only that CTA can wait on.  After a wait that ran out the two producers
+  // may have stopped at different stages (at most a ring apart): the first
+  // CTA settles each stage that only one of them issued (complete-tx for the
+  // copy that was announced but never made; expect-tx for a copy the second
+  // CTA made unannounced) and then waits, bounded, for the last phase of every
+  // slot, so that no copy is still in flight when either CTA leaves.  In a
+  // run without a timeout the two counts agree and every wait returns at once.
+  if (warp == 0 && lane == 0 && rank == 1)
+    st_cluster_u32(map_to_rank(smem_u32(&ctl->peer_issued), 0), ctl->issued);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both producers have stopped; the second one's count is posted
+  if (warp == 0 && lane == 0 && rank == 0) {
+    const uint32_t mine = ctl->issued, theirs = ctl->peer_issued;
+    const uint32_t hi = mine > theirs ? mine : theirs;
+    const uint32_t lo = hi > static_cast<uint32_t>(kStages) ? hi - kStages : 0u;
+    volatile int never = 0;
+    for (uint32_t q = lo; q < hi; ++q) {
+      uint64_t *bar = &ctl->full[q % kStages];
+      const uint32_t par = (q / kStages) & 1u;
+      if (q >= theirs) mbar_complete_tx(bar, kStageBytes);               // second CTA's share
+      if (q >= mine) mbar_arrive_expect_tx(bar, kStageBytes);            // only its copy
+      mbar_wait(bar, par, kDrainNs, &never);
     }
   }
-  tc_fence_before();
   __syncthreads();
   cluster_sync();  // neither CTA leaves while its peer may still touch it
   if (warp == 1) {
@@ -516,14 +540,9 @@ cudaError_t launch_w8a8_gemm(const int8_t *Xq, const int8_t *Wq, const float *x_
   a.group_m = 4;
   a.num_pairs = min(a.num_tiles, sm_count_of_current_device() / 2);
   a.timeout_ns = wait_timeout_ns();
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(w8a8_lora_gemm_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemBytes));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<int> attr_set[kMaxDevices];
+  const cudaError_t e = ensure_smem_optin(w8a8_lora_gemm_kernel, static_cast<int>(kSmemBytes), attr_set);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * a.num_pairs, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
