@@ -3,19 +3,34 @@
 
 One step = one pass of the whole hot path over one batch: sq_quant_act
 (smoothing + per-token INT8) followed by sq_linear_lora (LoRA shrink, then
-the fused INT8 GEMM + dequant + LoRA delta), on the Llama-3-8B fused QKV
-projection workload (M=2048 tokens, K=4096, N=6144, one rank-16 adapter).
+the fused INT8 GEMM + dequant + LoRA delta).
+
+The default run measures four workloads, one after another, in one process:
+the headline is the compute-bound down projection (M=16384 tokens, K=14336,
+N=4096, four rank-32 adapters over 64 request segments), the largest
+single-GPU workload; the fused QKV (M=2048, K=4096, N=6144, one rank-16
+adapter), the multi-tenant gate/up (M=8192, K=4096, N=28672, eight adapters
+over 32 segments) and the memory-bound decode step (M=64, K=4096, N=4096, 64
+rank-16 adapters, one per token) are reported beside it under "workloads",
+each with its own roofline, CPU baseline and end-to-end figure.
+`--workload NAME` measures one workload alone.
 
 Timing: W untimed warm-up steps, then K timed steps.  Before every step a
 256 MiB buffer is written and a second 256 MiB buffer is read (untimed), so
 that L2 (126 MB) holds none of the step's inputs and no dirty lines whose
-write-back would be charged to the step; each step is bracketed by CUDA events on the stream the
-kernels run on, and on every eighth timed step the fused GEMM launch also by
-its own event pair (recorded by the library; an event between the shrink and
-the GEMM keeps the GEMM from starting during the shrink's tail, ~8 us per
-step at the QKV shape, so it is not recorded on every step).  Multi-GPU runs are independent replicas (the layer has no
-exchange step): each rank runs the same workload, times are maxed over ranks
-and the throughput counts all ranks' work.
+write-back would be charged to the step; each step is bracketed by CUDA
+events on the stream the kernels run on, and on every eighth timed step the
+layer call's kernels also by their own event pair (recorded by the library;
+an event between the shrink and the GEMM keeps the GEMM from starting during
+the shrink's tail, so it is not recorded on every step).  Multi-GPU runs are
+independent replicas (the layer has no exchange step): each rank runs the
+same workload, times are maxed over ranks and the throughput counts all
+ranks' work.
+
+The decode workload is also run 1000 times back to back (a CUDA graph of
+steps, replayed), cycling through enough copies of Wq and the adapters that
+L2 cannot hold them between uses; its per-step latency is reported as
+"repeated".
 
 End to end (the "e2e" key): the same step through pinned host buffers, X
 copied in and Y copied out every step, with consecutive steps pipelined over
@@ -23,7 +38,8 @@ three streams (copy in, kernels, copy out) as a serving loop runs them; the
 serial form (one step at a time) is reported beside it.
 
 --impl reference times the CPU oracle (fp64/int64 C, OpenMP) on the host
-cores for the same workload and metric, one bounded sample of tokens per step.
+cores for the headline workload and metric, one bounded sample of tokens per
+step.
 """
 
 from __future__ import annotations
@@ -31,6 +47,7 @@ from __future__ import annotations
 import argparse
 import datetime
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -46,7 +63,7 @@ if ROOT not in sys.path:
 
 from w8a8_smoothquant_int8_b200 import workloads as wk  # noqa: E402
 
-GEMM_EVENT_EVERY = 8  # timed steps per step that also times the GEMM alone
+GEMM_EVENT_EVERY = 8  # timed steps per step that also times the layer's kernels alone
 # nominal figures, reported beside the measured denominators for context:
 # dense int8 tensor-core ops per SM per clock (4.5 POPS over 148 SMs near
 # 1.9 GHz) and the HBM3e bandwidth of the part
@@ -54,8 +71,15 @@ NOMINAL_INT8_OPS_PER_SM_CLK = 16384
 NOMINAL_HBM_GBS = 8000.0
 
 METRIC = "W8A8+LoRA linear INT8 TOPS & tokens/s; % of INT8 tensor peak / HBM roofline"
-DEFAULT_WORKLOAD = "llama3_8b_qkv_m2048_k4096_n6144"
+HEADLINE = "llama3_8b_down_m16384_k14336_n4096"
+BESIDE = ["llama3_8b_gateup_m8192_k4096_n28672", "llama3_8b_qkv_m2048_k4096_n6144",
+          "llama3_8b_oproj_decode_m64_k4096_n4096"]
 FLUSH_BYTES = 256 << 20
+DECODE_REPEAT = 1000
+# seconds of oracle work for the CPU baseline of the headline workload and of
+# each workload beside it (a bounded sample of its tokens)
+CPU_SECONDS_HEADLINE = 12.0
+CPU_SECONDS_BESIDE = 2.0
 
 
 def parse():
@@ -64,7 +88,8 @@ def parse():
     p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wk.SPECS))
+    p.add_argument("--workload", default="all", choices=["all"] + sorted(wk.SPECS),
+                   help="'all' (default): the headline workload and the three beside it")
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--act-quant", choices=["dynamic", "static"], default="dynamic",
@@ -80,27 +105,30 @@ def parse():
     return p.parse_args()
 
 
-# DRAM bytes (read + write) of one fused-GEMM launch on the default workload,
-# from the ncu capture summarised in profiles/w8a8_lora_gemm_llama3_8b_qkv_m2048.md.
-# It describes that kernel source only: any other source reports null.
-GEMM_TRAFFIC = {
-    "source_sha256": "c6429fb71707a01faa20e1b0b08fb3c3b2e7410a0fc50376fb111933d2470d6c",
-    "workload": DEFAULT_WORKLOAD,
-    "bytes": 34068992 + 1645824,
+# DRAM bytes (read + write) of one launch of the dominant kernel, per
+# workload, from an ncu capture of that kernel source (sha256 of the file that
+# holds it); any other source or workload reports null.
+KERNEL_TRAFFIC = {
+    "llama3_8b_qkv_m2048_k4096_n6144": {
+        "file": "gemm_sm100.cu",
+        "source_sha256": "c6429fb71707a01faa20e1b0b08fb3c3b2e7410a0fc50376fb111933d2470d6c",
+        "bytes": 34068992 + 1645824,
+    },
 }
 
 
-def gemm_traffic(workload: str):
+def kernel_traffic(workload: str):
     import hashlib
-    src = os.path.join(ROOT, "w8a8_smoothquant_int8_b200", "csrc", "gemm_sm100.cu")
+    ent = KERNEL_TRAFFIC.get(workload)
+    if ent is None:
+        return None
+    src = os.path.join(ROOT, "w8a8_smoothquant_int8_b200", "csrc", ent["file"])
     try:
         with open(src, "rb") as f:
             sha = hashlib.sha256(f.read()).hexdigest()
     except OSError:
         return None
-    if sha != GEMM_TRAFFIC["source_sha256"] or workload != GEMM_TRAFFIC["workload"]:
-        return None
-    return GEMM_TRAFFIC["bytes"]
+    return ent["bytes"] if sha == ent["source_sha256"] else None
 
 
 def measured_peaks():
@@ -123,6 +151,12 @@ def decode_layer_bytes(wl) -> int:
     used = sorted(set(int(a) for a in ad if a >= 0))
     lora = sum(2 * wl.adapters[a].r * (wl.K + wl.N) for a in used)
     return int(wl.N * wl.K + 4 * wl.N + wl.M * wl.K + 4 * wl.M + lora + 2 * wl.M * wl.N)
+
+
+def quant_bytes(wl) -> int:
+    """Algorithmic HBM bytes of sq_quant_act: X read, codes and scales written."""
+    xb = 2 if wl.x_is_bf16 else 4
+    return int(wl.M * wl.K * (xb + 1) + 4 * wl.M + 4 * wl.K)
 
 
 def lora_flops(wl) -> int:
@@ -225,17 +259,27 @@ def oracle_step(P, wl, rows, raw=False):
         oracle.linear_lora_rows(Xq, xs, P.Wq, P.w_scale, P.A_s, P.B_s, so, sa, want=("Y",))
 
 
-def cpu_baseline(wl, sample_rows=None, raw=False):
+def cpu_baseline(wl, seconds: float, raw=False):
+    """The oracle over a bounded sample of the workload's tokens: a 16-token
+    probe sizes the sample to about `seconds` of work (the whole workload if
+    it is shorter), then the sample is timed in one pass."""
     import oracle
     P = oracle.Prepared(wl)
-    rows = np.arange(wl.M if sample_rows is None else min(sample_rows, wl.M))
+    probe = np.arange(min(16, wl.M))
+    t0 = time.perf_counter()
+    oracle_step(P, wl, probe, raw)
+    t_probe = max(time.perf_counter() - t0, 1e-6)
+    n = int(min(wl.M, max(len(probe), len(probe) * seconds / t_probe)))
+    rows = np.sort(np.random.default_rng(0).choice(wl.M, size=n, replace=False)) \
+        if n < wl.M else np.arange(wl.M)
     t0 = time.perf_counter()
     oracle_step(P, wl, rows, raw)
     dt = time.perf_counter() - t0
     ops = 2 * len(rows) * wl.N * wl.K
+    what = "all" if n == wl.M else f"{n} random"
     return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": oracle.num_threads(),
             "kind": "oracle",
-            "sample": f"{len(rows)} of {wl.M} tokens, whole hot path (quantize, int64 GEMM, fp64 "
+            "sample": f"{what} of {wl.M} tokens, whole hot path (quantize, int64 GEMM, fp64 "
                       f"dequant + LoRA on the {'raw activations' if raw else 'dequantized codes'}), "
                       f"one pass, {dt:.2f} s",
             "tokens_per_s": len(rows) / dt}
@@ -246,9 +290,10 @@ def run_reference(args):
     if rank != 0:
         return 0
     import oracle
-    wl = wk.make_workload(args.workload)
+    name = HEADLINE if args.workload == "all" else args.workload
+    wl = wk.make_workload(name)
     P = oracle.Prepared(wl)
-    sample = min(wl.M, 256)
+    sample = min(wl.M, 64)
     rng = np.random.default_rng(0)
     times = []
     for i in range(args.warmup + args.steps):
@@ -281,28 +326,18 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # GPU path
 # ---------------------------------------------------------------------------
-def run_ours(args):
+def measure(name, args, dev, world, local_rank, cpu_seconds):
+    """Time one workload; returns its entry (value, roofline, e2e, ...)."""
     import torch
     import torch.distributed as dist
 
     import w8a8_smoothquant_int8_b200 as sq
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=dev)
-    if sq.sq_device_supported(local_rank) != 0:
-        raise SystemExit("device is not compute capability 10.0")
-
-    # cpu baseline first (rank 0, N=1 only), before any CUDA work in this process
-    wl = wk.make_workload(args.workload)
+    wl = wk.make_workload(name)
+    raw = args.lora_input == "raw"
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, raw=args.lora_input == "raw")
+    if cpu_seconds > 0:
+        cpu = cpu_baseline(wl, cpu_seconds, raw=raw)
 
     M, K, N = wl.M, wl.K, wl.N
 
@@ -325,7 +360,6 @@ def run_ours(args):
     w_scale = torch.empty(N, dtype=torch.float32, device=dev)
     sq.sq_quantize_weight(W, s, Wq, w_scale)
     del W
-    raw = args.lora_input == "raw"
     if raw and not wl.x_is_bf16:
         raise SystemExit("--lora-input raw needs bf16 activations")
     lora = sq.LoraPack.build([h2d(a.A) for a in wl.adapters], [h2d(a.B) for a in wl.adapters],
@@ -359,7 +393,9 @@ def run_ours(args):
         sq.sq_static_act_scale(act_absmax, s, static_scale)
         clip_count = torch.zeros(1, dtype=torch.int64, device=dev)
 
-    def step(Xb=X, Yb=Y):
+    decode = M <= DECODE_MAX_M and not raw
+
+    def step(Xb=X, Yb=Y, Wqb=Wq, wsb=w_scale, lorab=lora):
         if norm:
             sq.sq_rmsnorm_quant_act(Xb, gamma_s, 1e-6, Xq, x_scale)
         elif static:
@@ -367,12 +403,12 @@ def run_ours(args):
         else:
             sq.sq_quant_act(Xb, s, Xq, x_scale)
         if raw:
-            sq.sq_lora_shrink_raw(Xb, lora, seg_offsets, seg_adapter, ws)
-            sq.sq_linear_lora_from_t(Xq, x_scale, Wq, w_scale, lora, Yb, ws)
+            sq.sq_lora_shrink_raw(Xb, lorab, seg_offsets, seg_adapter, ws)
+            sq.sq_linear_lora_from_t(Xq, x_scale, Wqb, wsb, lorab, Yb, ws)
         else:
-            sq.sq_linear_lora(Xq, x_scale, Wq, w_scale, lora, seg_offsets, seg_adapter, Yb, ws)
+            sq.sq_linear_lora(Xq, x_scale, Wqb, wsb, lorab, seg_offsets, seg_adapter, Yb, ws)
 
-    launches_per_step = 3  # quantize, LoRA shrink, fused GEMM
+    launches_per_step = 3  # quantize, LoRA shrink, fused GEMM (or the decode pair)
 
     sampler = ClockSampler(local_rank)
     sampler.start()
@@ -391,10 +427,10 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    # the GEMM's own event pair sits between the shrink and the GEMM in the
-    # stream and keeps the GEMM from starting during the shrink's tail, so it
-    # is recorded on every GEMM_EVENT_EVERY-th timed step only (all K steps
-    # count towards the step time)
+    # the layer call's own event pair sits between the quantizer and the
+    # shrink, and between the shrink and the GEMM; recorded on every
+    # GEMM_EVENT_EVERY-th timed step only (all K steps count towards the step
+    # time)
     gemm_steps = [i for i in range(n) if i % GEMM_EVENT_EVERY == GEMM_EVENT_EVERY // 2]
     gemm_steps = gemm_steps or [n // 2]
     for i in range(n):
@@ -416,6 +452,54 @@ def run_ours(args):
     err = sq.sq_get_device_error(clear=True)
     if err:
         raise SystemExit(f"device error {err}: {sq.sq_status_string(err)}")
+
+    # decode: 1000 steps back to back in a CUDA graph, cycling through copies
+    # of Wq, w_scale and the adapters so that none is still in L2 when it is
+    # used again (copies x bytes >= 4 x L2)
+    repeated = None
+    if decode:
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        copies = max(2, math.ceil(4 * l2 / decode_layer_bytes(wl)))
+        reps = [(Wq, w_scale, lora)]
+        for _ in range(copies - 1):
+            lp = sq.LoraPack(lora.A_pack.clone(), lora.B_pack.clone(), lora.offset.clone(),
+                             lora.rank.clone(), lora.R, lora.n_adapters)
+            reps.append((Wq.clone(), w_scale.clone(), lp))
+        g_stream = torch.cuda.Stream(dev)
+        g_stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(g_stream):
+            for r in reps:  # warm: the library's first call per device does its set-up
+                step(Wqb=r[0], wsb=r[1], lorab=r[2])
+        g_stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=g_stream):
+            for r in reps:
+                step(Wqb=r[0], wsb=r[1], lorab=r[2])
+        replays = math.ceil(DECODE_REPEAT / copies)
+        for _ in range(2):
+            graph.replay()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(replays):
+            graph.replay()
+        b.record()
+        torch.cuda.synchronize()
+        t_rep = reduce_max([a.elapsed_time(b)], dev)[0]
+        steps_rep = replays * copies
+        us = 1e3 * t_rep / steps_rep
+        step_bytes = decode_layer_bytes(wl) + quant_bytes(wl)
+        repeated = {"steps": steps_rep, "us_per_step": us,
+                    "tokens_per_s": M * steps_rep * world / (t_rep * 1e-3),
+                    "step_bytes": step_bytes, "gbs": step_bytes / (us * 1e-6) / 1e9,
+                    "form": f"CUDA graph of {copies} steps (one per copy of Wq, w_scale and the "
+                            f"adapters, {copies} x {decode_layer_bytes(wl) / 1e6:.1f} MB), "
+                            f"replayed {replays} times; inputs not flushed between steps"}
+        del graph, reps
+        err = sq.sq_get_device_error(clear=True)
+        if err:
+            raise SystemExit(f"device error {err}: {sq.sq_status_string(err)}")
 
     # end to end through the public API with host buffers: every step copies
     # its X in from pinned host memory and its Y out to pinned host memory.
@@ -481,28 +565,29 @@ def run_ours(args):
 
     e2e = None
     n_e2e = args.e2e_steps
+    ops_step = 2 * M * N * K
     if n_e2e > 0:
-        e2e_serial(args.warmup)
+        e2e_serial(min(args.warmup, 3))
         t_serial = reduce_max([e2e_serial(n_e2e)], dev)[0]
-        e2e_pipelined(max(args.warmup, 2))
+        e2e_pipelined(max(min(args.warmup, 3), 2))
         t_e2e = reduce_max([e2e_pipelined(n_e2e)], dev)[0]
-        e2e = {"value": job_tops(2 * M * N * K, n_e2e, world, t_e2e), "unit": "TOPS",
+        e2e = {"value": job_tops(ops_step, n_e2e, world, t_e2e), "unit": "TOPS",
                "h2d_bytes_per_step": int(X_host.numel() * X_host.element_size()),
                "d2h_bytes_per_step": int(Y_host.numel() * Y_host.element_size()),
                "ms_per_step": t_e2e / n_e2e,
+               "tokens_per_s": M * n_e2e * world / (t_e2e * 1e-3),
                "form": "pipelined: copy in, kernels and copy out of consecutive steps "
                        "on three streams (two device buffers for X and Y)",
-               "serial": {"value": job_tops(2 * M * N * K, n_e2e, world, t_serial),
+               "serial": {"value": job_tops(ops_step, n_e2e, world, t_serial),
                           "ms_per_step": t_serial / n_e2e}}
 
-    ops_step = 2 * M * N * K
     value = job_tops(ops_step, n, world, t_step_total)
     tok_s = M * n * world / (t_step_total * 1e-3)
     gemm_avg_s = t_gemm_total * 1e-3 / max(1, len(gemm_steps))
     gemm_tops = ops_step / gemm_avg_s / 1e12
     peaks, peak_kind = measured_peaks()
     int8_peak = 2.0 * float(peaks["bf16_tflops"])  # dense int8 = 2x dense bf16 (nominal ratio)
-    if M <= DECODE_MAX_M and not raw:
+    if decode:
         # decode form: bound by streaming Wq and the adapters from HBM; the
         # timed region is the whole layer call (shrink + GEMM kernels)
         nbytes = decode_layer_bytes(wl)
@@ -512,8 +597,8 @@ def run_ours(args):
                     "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                     "peak_source": f"{peak_kind}: copy bandwidth {hbm} GB/s",
                     "frac_of_nominal": gbs / NOMINAL_HBM_GBS,
-                    "layer_us": gemm_avg_s * 1e6, "traffic": None,
-                    "traffic_unit": "bytes per launch (ncu dram read+write)",
+                    "layer_us": gemm_avg_s * 1e6, "traffic": kernel_traffic(wl.spec.name),
+                    "traffic_unit": "bytes per layer call (ncu dram read+write, both kernels)",
                     "algorithmic_bytes": nbytes}
     else:
         # context: the nominal dense int8 rate at the SM clock sampled under load
@@ -525,22 +610,14 @@ def run_ours(args):
                     "peak_source": f"{peak_kind}: 2 x bf16 burst {peaks['bf16_tflops']} TFLOP/s",
                     "clock_normalized_peak": clk_peak or None,
                     "frac_of_clock_normalized": (gemm_tops / clk_peak) if clk_peak else None,
-                    "gemm_us": gemm_avg_s * 1e6, "traffic": gemm_traffic(wl.spec.name),
+                    "gemm_us": gemm_avg_s * 1e6, "traffic": kernel_traffic(wl.spec.name),
                     "traffic_unit": "bytes per launch (ncu dram read+write)",
                     "algorithmic_ops": ops_step}
-    line = {
-        "metric": METRIC,
+    entry = {
         "value": value,
         "unit": "TOPS",
-        "n_gpus": world,
-        "steps": n,
-        "warmup": args.warmup,
         "ms_per_step": t_step_total / n,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "int8",
-        "data": "synthetic",
+        "tokens_per_s": tok_s,
         "config": {"workload": wl.spec.name, "M": M, "K": K, "N": N,
                    "adapters": len(wl.adapters), "ranks": sorted(set(a.r for a in wl.adapters)),
                    "segments": int(len(wl.seg_adapter)), "alpha": wl.alpha,
@@ -552,7 +629,6 @@ def run_ours(args):
                    "act_quant": args.act_quant,
                    "l2": "flushed between timed steps (256 MiB write + 256 MiB read, untimed)",
                    "parallelism": f"replicas x{world}"},
-        "tokens_per_s": tok_s,
         "lora_flops_per_step": lora_flops(wl),
         "roofline": roofline,
         "cpu_baseline": cpu,
@@ -560,6 +636,67 @@ def run_ours(args):
         "clocks": clocks,
         "gpu_launches": launches_per_step * n * world,
     }
+    if repeated is not None:
+        entry["repeated"] = repeated
+    return entry
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import w8a8_smoothquant_int8_b200 as sq
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    if sq.sq_device_supported(local_rank) != 0:
+        raise SystemExit("device is not compute capability 10.0")
+
+    with_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    if args.workload == "all":
+        head, beside = HEADLINE, BESIDE
+    else:
+        head, beside = args.workload, []
+
+    entries = {}
+    for name in [head] + beside:
+        secs = (CPU_SECONDS_HEADLINE if name == head else CPU_SECONDS_BESIDE) if with_cpu else 0.0
+        entries[name] = measure(name, args, dev, world, local_rank, secs)
+        torch.cuda.empty_cache()
+
+    h = entries[head]
+    line = {
+        "metric": METRIC,
+        "value": h["value"],
+        "unit": "TOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": h["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8",
+        "data": "synthetic",
+        "config": h["config"],
+        "tokens_per_s": h["tokens_per_s"],
+        "lora_flops_per_step": h["lora_flops_per_step"],
+        "roofline": h["roofline"],
+        "cpu_baseline": h["cpu_baseline"],
+        "e2e": h["e2e"],
+        "clocks": h["clocks"],
+        "gpu_launches": h["gpu_launches"],
+    }
+    if "repeated" in h:
+        line["repeated"] = h["repeated"]
+    if beside:
+        line["workloads"] = {name: entries[name] for name in beside}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

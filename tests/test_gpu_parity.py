@@ -17,7 +17,8 @@ pytestmark = pytest.mark.gpu
 Y_TOL = 1e-2
 DELTA_TOL = 5e-3
 
-SMALL = ["tiny_m16_k256_n256", "parity_ragged", "parity_heavy_f32", "parity_decode"]
+SMALL = ["tiny_m16_k256_n256", "parity_ragged", "parity_heavy_f32", "parity_decode",
+         "parity_waves"]
 
 
 def _run(name, **kw):
@@ -103,8 +104,11 @@ FULL = ["llama3_8b_qkv_m2048_k4096_n6144", "llama3_8b_gateup_m8192_k4096_n28672"
 
 
 def _sample_rows(M, rng, n=24):
+    # tile edges, random rows, and one random row of every 256-row tile
     rows = {0, M - 1, min(127, M - 1), min(128, M - 1)}
     rows |= set(rng.choice(M, size=min(M, n), replace=False).tolist())
+    for t0 in range(0, M, 256):
+        rows.add(int(rng.integers(t0, min(M, t0 + 256))))
     return np.array(sorted(rows), np.int64)
 
 
@@ -117,6 +121,7 @@ def test_full_size_sampled(name):
     assert np.array_equal(g.x_scale.cpu().numpy().view(np.uint32), P.x_scale.view(np.uint32))
     assert np.array_equal(g.Xq.cpu().numpy(), P.Xq)
     assert np.array_equal(g.Wq.cpu().numpy(), P.Wq)
+    assert np.array_equal(g.w_scale.cpu().numpy().view(np.uint32), P.w_scale.view(np.uint32))
     rows = _sample_rows(wl.M, rng)
     out = P.rows(rows)
     acc = g.gemm_i32()

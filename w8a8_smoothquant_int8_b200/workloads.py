@@ -104,6 +104,14 @@ SPECS = {
     "parity_decode": WorkloadSpec(
         "parity_decode", 64, 1024, 512, "bf16", "normal", 5, 50.0, 50.0,
         0.5, 128, (16,) * 64, "per_token", 64),
+    # more than four waves of 256x256 output tiles on 74 CTA pairs (9 x 36 =
+    # 324 tiles, the last row and column ragged), a ragged K tail, four
+    # adapters of different ranks and segments without an adapter: the
+    # persistent schedule, the double-buffered accumulators and the deferred
+    # LoRA MMAs all run, and the oracle still checks every element in seconds
+    "parity_waves": WorkloadSpec(
+        "parity_waves", 2300, 272, 9200, "bf16", "normal", 6, 20.0, 100.0,
+        0.5, 256, (8, 16, 64, 32), "random", 9, 0.2),
 }
 
 # benchmark workloads in the order they are listed with the benchmark
