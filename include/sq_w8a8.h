@@ -149,6 +149,27 @@ int sq_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s, int64_
                     int64_t K, int64_t N, float lora_alpha, int64_t R, int64_t off,
                     uint16_t *A_pack, uint16_t *B_pack, void *stream);
 
+/* The whole adapter table in one call, from adapters held in separate
+ * buffers (a list lora_A[], lora_B[] of per-request adapters, "[Feature]:
+ * LoRA support for W8A8 SmoothQuant", Motivation: one adapter per request).
+ * A[a] [ranks[a], K] and B[a] [N, ranks[a]] (bf16, device) are given as host
+ * arrays of n_adapters device pointers, with lora_alpha[a] (host) and s
+ * (device; NULL packs A unchanged, as sq_prepare_lora).  Adapter a goes to
+ * columns [off_a, off_a + round_up(r_a, 16)), off_a the sum of the earlier
+ * adapters' rounded ranks; R must be that total (sq_lora_pack_width).
+ * Writes A_pack [R, K], B_pack [N, R] as sq_prepare_lora does for each
+ * adapter, and lora_offset, lora_rank [n_adapters] (device int32) = off_a,
+ * r_a: the table sq_linear_lora takes.  Errors: SQ_ERR_INVALID_ARG (null or
+ * misaligned pointers, a rank outside [1, SQ_MAX_LORA_RANK], R not the
+ * total), SQ_ERR_UNSUPPORTED_SHAPE (K % 16, K > SQ_MAX_K, total width above
+ * SQ_MAX_LORA_COLS).  Enqueued on `stream`; the host arrays may be reused
+ * when the call returns. */
+int64_t sq_lora_pack_width(const int64_t *ranks, int n_adapters);
+int sq_pack_lora(const uint16_t *const *A, const uint16_t *const *B, const int64_t *ranks,
+                 const float *lora_alpha, int n_adapters, const float *s, int64_t K, int64_t N,
+                 int64_t R, uint16_t *A_pack, uint16_t *B_pack, int32_t *lora_offset,
+                 int32_t *lora_rank, void *stream);
+
 /* ---------------------------------------------------------------------------
  * Hot path
  * ------------------------------------------------------------------------ */

@@ -62,6 +62,9 @@ def test_lora_pack_bit_exact(small):
     B_pack = bf16_bits(g.lora.B_pack)
     offs, R = g.lora.layout([a.r for a in wl.adapters])
     assert g.lora.R == R
+    # the table written by sq_pack_lora
+    assert g.lora.offset.cpu().tolist() == offs
+    assert g.lora.rank.cpu().tolist() == [a.r for a in wl.adapters]
     for a, off in enumerate(offs):
         r = wl.adapters[a].r
         rpad = (r + 15) // 16 * 16

@@ -20,7 +20,8 @@ from . import _native
 __all__ = [
     "SQError", "LoraPack", "sq_status_string", "sq_version", "sq_device_supported",
     "sq_get_device_error", "sq_set_wait_timeout_ns", "sq_set_gemm_events", "sq_selftest_wait_timeout", "sq_act_absmax_update", "sq_weight_absmax",
-    "sq_compute_smoothing", "sq_quantize_weight", "sq_prepare_lora", "sq_quant_act",
+    "sq_compute_smoothing", "sq_quantize_weight", "sq_prepare_lora", "sq_lora_pack_width",
+    "sq_pack_lora", "sq_quant_act",
     "sq_linear_lora_workspace_size", "sq_linear_lora", "sq_linear_lora_noalloc", "sq_gemm_i32",
     "sq_lora_delta", "sq_lora_t_workspace_size", "sq_lora_shrink_raw", "sq_linear_lora_from_t",
     "sq_lora_delta_from_t", "sq_static_act_scale", "sq_quant_act_static",
@@ -131,6 +132,27 @@ def sq_quantize_weight(W, s, Wq, w_scale, stream=None) -> None:
            "sq_quantize_weight")
 
 
+def sq_lora_pack_width(ranks: Sequence[int]) -> int:
+    arr = (ctypes.c_int64 * max(1, len(ranks)))(*[int(r) for r in ranks])
+    return int(_lib().sq_lora_pack_width(arr, len(ranks)))
+
+
+def sq_pack_lora(As: List, Bs: List, lora_alphas: Sequence[float], s, R: int, A_pack, B_pack,
+                 lora_offset, lora_rank, stream=None) -> None:
+    """Every adapter (A [r,K], B [N,r] bf16 device tensors) into one pack and
+    its offset/rank tables (sq_pack_lora)."""
+    n = len(As)
+    K = As[0].shape[1]
+    N = Bs[0].shape[0]
+    pa = (ctypes.c_void_p * n)(*[_ptr(a) for a in As])
+    pb = (ctypes.c_void_p * n)(*[_ptr(b) for b in Bs])
+    rk = (ctypes.c_int64 * n)(*[int(a.shape[0]) for a in As])
+    al = (ctypes.c_float * n)(*[float(x) for x in lora_alphas])
+    _check(_lib().sq_pack_lora(pa, pb, rk, al, n, _ptr(s), K, N, int(R), _ptr(A_pack),
+                               _ptr(B_pack), _ptr(lora_offset), _ptr(lora_rank), _stream(stream)),
+           "sq_pack_lora")
+
+
 def sq_prepare_lora(A, B, s, lora_alpha: float, R: int, off: int, A_pack, B_pack, stream=None) -> None:
     r, K = A.shape
     N = B.shape[0]
@@ -196,7 +218,7 @@ class LoraPack:
 
     @classmethod
     def build(cls, As: List, Bs: List, lora_alphas: Sequence[float], s, stream=None) -> "LoraPack":
-        """Pack adapters (A [r,K], B [N,r] bf16 device tensors) with sq_prepare_lora.
+        """Pack adapters (A [r,K], B [N,r] bf16 device tensors) with sq_pack_lora.
 
         s=None packs A unchanged, for the raw-input entry points
         (sq_lora_shrink_raw / sq_linear_lora_from_t)."""
@@ -204,14 +226,14 @@ class LoraPack:
         K = s.shape[0] if s is not None else As[0].shape[1]
         N = Bs[0].shape[0] if Bs else 0
         ranks = [a.shape[0] for a in As]
-        offs, R = cls.layout(ranks)
+        _, R = cls.layout(ranks)
         dev = s.device if s is not None else As[0].device
         A_pack = torch.empty((max(R, 1), K), dtype=torch.bfloat16, device=dev)
         B_pack = torch.empty((max(N, 1), max(R, 1)), dtype=torch.bfloat16, device=dev)
-        for A, B, la, off in zip(As, Bs, lora_alphas, offs):
-            sq_prepare_lora(A, B, s, la, R, off, A_pack, B_pack, stream)
-        offset = torch.tensor(offs or [0], dtype=torch.int32, device=dev)
-        rank = torch.tensor(ranks or [0], dtype=torch.int32, device=dev)
+        offset = torch.zeros(max(1, len(ranks)), dtype=torch.int32, device=dev)
+        rank = torch.zeros(max(1, len(ranks)), dtype=torch.int32, device=dev)
+        if ranks:
+            sq_pack_lora(As, Bs, lora_alphas, s, R, A_pack, B_pack, offset, rank, stream)
         return cls(A_pack, B_pack, offset, rank, R, len(ranks))
 
 

@@ -32,6 +32,8 @@ SIGNATURES = {
     "sq_compute_smoothing": ([P, P, I64, F32, P, P], I32),
     "sq_quantize_weight": ([P, P, I64, I64, P, P, P], I32),
     "sq_prepare_lora": ([P, P, P, I64, I64, I64, F32, I64, I64, P, P, P], I32),
+    "sq_lora_pack_width": ([P, I32], I64),
+    "sq_pack_lora": ([P, P, P, P, I32, P, I64, I64, I64, P, P, P, P, P], I32),
     "sq_quant_act": ([P, I32, P, I64, I64, P, P, P], I32),
     "sq_linear_lora_workspace_size": ([I64, I64], SZ),
     "sq_linear_lora": ([P, P, P, P, I64, I64, I64, P, P, P, P, I32, I64, P, P, I64, P, P, SZ, P],

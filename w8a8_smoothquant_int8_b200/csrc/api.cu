@@ -17,6 +17,9 @@ uint64_t wait_timeout_ns() { return g_wait_timeout_ns; }
 // ---------------------------------------------------------------------------
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 static bool ptr_ok(const void *p) { return p != nullptr && aligned16(p); }
+static bool aligned_to(const void *p, uintptr_t a) {
+  return p != nullptr && (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
 
 // Result of sq_device_supported per device, cached: querying the device
 // properties takes far longer than a launch.
@@ -237,6 +240,49 @@ int sq_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s, int64_
                                          static_cast<cudaStream_t>(stream)));
 }
 
+int64_t sq_lora_pack_width(const int64_t *ranks, int n_adapters) {
+  if (!ranks || n_adapters < 1) return -1;
+  int64_t R = 0;
+  for (int a = 0; a < n_adapters; ++a) {
+    if (ranks[a] < 1 || ranks[a] > SQ_MAX_LORA_RANK) return -1;
+    R += (ranks[a] + 15) / 16 * 16;
+  }
+  return R;
+}
+
+int sq_pack_lora(const uint16_t *const *A, const uint16_t *const *B, const int64_t *ranks,
+                 const float *lora_alpha, int n_adapters, const float *s, int64_t K, int64_t N,
+                 int64_t R, uint16_t *A_pack, uint16_t *B_pack, int32_t *lora_offset,
+                 int32_t *lora_rank, void *stream) {
+  if (!A || !B || !ranks || !lora_alpha || n_adapters < 1 || K < 0 || N < 0)
+    return SQ_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K > SQ_MAX_K) return SQ_ERR_UNSUPPORTED_SHAPE;
+  const int64_t width = sq_lora_pack_width(ranks, n_adapters);
+  if (width < 0) return SQ_ERR_INVALID_ARG;
+  if (width > SQ_MAX_LORA_COLS) return SQ_ERR_UNSUPPORTED_SHAPE;
+  if (R != width) return SQ_ERR_INVALID_ARG;
+  if ((s && !ptr_ok(s)) || !ptr_ok(A_pack) || !ptr_ok(B_pack) || !aligned_to(lora_offset, 4) ||
+      !aligned_to(lora_rank, 4))
+    return SQ_ERR_INVALID_ARG;
+  for (int a = 0; a < n_adapters; ++a)
+    if (!A[a] || !B[a]) return SQ_ERR_INVALID_ARG;
+  int st = check_device();
+  if (st) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int32_t offs[SQ_MAX_LORA_COLS / 16], rks[SQ_MAX_LORA_COLS / 16];
+  int64_t off = 0;
+  for (int a = 0; a < n_adapters; ++a) {
+    const float scale = lora_alpha[a] / static_cast<float>(ranks[a]);  // IEEE fp32 division
+    cudaError_t e = launch_prepare_lora(A[a], B[a], s, ranks[a], K, N, scale, R, off, A_pack,
+                                        B_pack, cs);
+    if (e != cudaSuccess) return SQ_ERR_CUDA;
+    offs[a] = static_cast<int32_t>(off);
+    rks[a] = static_cast<int32_t>(ranks[a]);
+    off += (ranks[a] + 15) / 16 * 16;
+  }
+  return cuda_status(launch_write_lora_table(offs, rks, n_adapters, lora_offset, lora_rank, cs));
+}
+
 int sq_quant_act(const void *X, int x_dtype, const float *s, int64_t M, int64_t K, int8_t *Xq,
                  float *x_scale, void *stream) {
   int st = check_mk(M, K);
@@ -249,9 +295,6 @@ int sq_quant_act(const void *X, int x_dtype, const float *s, int64_t M, int64_t 
       launch_quant_act(X, x_dtype, s, M, K, Xq, x_scale, static_cast<cudaStream_t>(stream)));
 }
 
-static bool aligned_to(const void *p, uintptr_t a) {
-  return p != nullptr && (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
-}
 
 int sq_static_act_scale(const float *act_absmax, const float *s, int64_t K, float *scale,
                         void *stream) {

@@ -114,6 +114,8 @@ cudaError_t launch_quantize_weight(const uint16_t *W, const float *s, int64_t N,
 cudaError_t launch_prepare_lora(const uint16_t *A, const uint16_t *B, const float *s, int64_t r,
                                 int64_t K, int64_t N, float scale, int64_t R, int64_t off,
                                 uint16_t *A_pack, uint16_t *B_pack, cudaStream_t st);
+cudaError_t launch_write_lora_table(const int32_t *offs, const int32_t *ranks, int n,
+                                    int32_t *off_dev, int32_t *rank_dev, cudaStream_t st);
 cudaError_t launch_lora_shrink(const int8_t *Xq, const float *x_scale, int64_t M, int64_t K,
                                const uint16_t *A_pack, const int32_t *lora_offset,
                                const int32_t *lora_rank, int n_adapters, int64_t R,

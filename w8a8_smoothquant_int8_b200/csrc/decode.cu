@@ -126,7 +126,11 @@ __device__ void decode_lookup(const int32_t *__restrict__ seg_offsets,
 // Thread t covers 8 consecutive K elements per pass and loads the 16 A' rows
 // of a rank group together (all of the block's 16 x 4 KB at once).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kDecShrinkThreads, 2) decode_shrink_kernel(
+// At most 104 registers a thread: an SM's registers are split between its
+// four sub-partitions (16K each) and a block's warps are dealt to them in
+// turn, so a GEMM CTA (9 warps of 96 registers: 3 on one sub-partition) fits
+// beside a shrink block (2 warps on each) only while 3*96 + 2*r <= 512.
+__global__ void __maxnreg__(104) decode_shrink_kernel(
     const int8_t *__restrict__ Xq, int64_t M, int64_t K, int ksplit,
     const uint16_t *__restrict__ A_pack, const int32_t *__restrict__ lora_offset,
     const int32_t *__restrict__ lora_rank, int n_adapters, int64_t R,
@@ -254,10 +258,15 @@ struct DecodeCtl {
   DecodeTables tb;
   int abort;
   int bdense;                      // B' rows staged in shared memory (first tile)
+  int rmax;                        // largest rank among the tokens
 };
 // after the K loop the ring holds the int32 partials [64][64] and then T [64][256] fp32
-constexpr int kDecPartBytes = kDecMaxM * kDecRowsMax * 4;
-static_assert(kDecPartBytes + kDecMaxM * kDecMaxRank * 4 <= kDecStages * kDecStageBytes,
+// (row strides padded so that the epilogue's lanes, which walk tokens, hit
+// distinct shared-memory banks)
+constexpr int kDecPStride = kDecRowsMax + 2;         // int32 per partial row
+constexpr int kDecTStride = kDecMaxRank + 4;         // fp32 per T row
+constexpr int kDecPartBytes = (kDecMaxM * kDecPStride * 4 + 15) / 16 * 16;
+static_assert(kDecPartBytes + kDecMaxM * kDecTStride * 4 <= kDecStages * kDecStageBytes,
               "partials and T must fit the ring");
 
 constexpr size_t kDecSmemBytes =
@@ -300,8 +309,8 @@ __global__ void __launch_bounds__(kDecGemmThreads, 2) decode_gemm_kernel(
                                               ~static_cast<uintptr_t>(1023));
   uint16_t *bsm = reinterpret_cast<uint16_t *>(ring + kDecStages * kDecStageBytes);
   DecodeCtl &ctl = *reinterpret_cast<DecodeCtl *>(ring + kDecStages * kDecStageBytes + kDecBBytes);
-  int *P = reinterpret_cast<int *>(ring);                          // [64][64] int32
-  float *Tm = reinterpret_cast<float *>(ring + kDecPartBytes);     // [64][256] fp32
+  int *P = reinterpret_cast<int *>(ring);                          // [64][kDecPStride] int32
+  float *Tm = reinterpret_cast<float *>(ring + kDecPartBytes);     // [64][kDecTStride] fp32
   volatile int *abort_flag = &ctl.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t crank = cluster_ctarank();
@@ -314,6 +323,9 @@ __global__ void __launch_bounds__(kDecGemmThreads, 2) decode_gemm_kernel(
   const int kb0 = static_cast<int>(crank) * nk_half;
   const int my_nk = max(0, min(nk, kb0 + nk_half) - kb0);
   const int nstage = (my_nk + kDecKbStage - 1) / kDecKbStage;
+  // the pairs start their K walk at different stages, so that few CTAs read
+  // the same Xq lines of L2 at once
+  const int rot = nstage > 0 ? pair % nstage : 0;
   const int mt = static_cast<int>(min(M, static_cast<int64_t>(kDecMaxM)));
 
   if (threadIdx.x == 0) {
@@ -366,7 +378,8 @@ __global__ void __launch_bounds__(kDecGemmThreads, 2) decode_gemm_kernel(
       for (int si = 0; si < nstage; ++si) {
         const int slot = q % kDecStages;
         const uint32_t ph = static_cast<uint32_t>(q / kDecStages) & 1u;
-        const int kbs = kb0 + si * kDecKbStage;                       // first K block
+        const int sj = si + rot < nstage ? si + rot : si + rot - nstage;
+        const int kbs = kb0 + sj * kDecKbStage;                       // first K block
         const int nkb = min(kDecKbStage, kb0 + my_nk - kbs);          // this CTA's blocks
         const int boxes = view3d ? kDecKbStage : nkb;                 // K blocks copied
         bool got = true;
@@ -439,6 +452,12 @@ __global__ void __launch_bounds__(kDecGemmThreads, 2) decode_gemm_kernel(
     for (int i = tid; i < kDecMaxM; i += kDecComputeThreads) ctl.tok_rank[i] = 0;
   for (int i = tid; i < kDecMaxM; i += kDecComputeThreads)
     ctl.xs[i] = (mode != 1 && i < M) ? __ldg(x_scale + i) : 0.f;
+  if (warp == 0) {  // (the lookup ended with a barrier of the compute warps)
+    int r = max(lane < mt ? ctl.tok_rank[lane] : 0, lane + 32 < mt ? ctl.tok_rank[lane + 32] : 0);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) r = max(r, __shfl_xor_sync(0xffffffffu, r, o));
+    if (lane == 0) ctl.rmax = r;
+  }
   group_bar(kBarLookup, kDecGemmThreads);
 
   const int mtile = warp & 3, ng = warp >> 2;
@@ -448,13 +467,15 @@ __global__ void __launch_bounds__(kDecGemmThreads, 2) decode_gemm_kernel(
   for (int tile = pair; tile < tiles; tile += npairs) {
     const int64_t n0 = static_cast<int64_t>(tile) * tile_rows;
     const int64_t c0 = n0 + static_cast<int64_t>(crank) * half;  // this CTA's first channel
-    const int tok = tid >> 2;                                       // epilogue token
+    // epilogue: token tok = tid % 64 and channel pairs p = tid/64 + 4m of this
+    // CTA's half of the tile (a warp's lanes walk 32 tokens)
+    const int tok = tid & 63;
     const int npairs_out = half / 2;
     // w_scale of this thread's epilogue channels, loaded ahead of every wait
     float wsv[4][2];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-      const int p = (tid & 3) + 4 * m;
+      const int p = (tid >> 6) + 4 * m;
       const int64_t n = c0 + 2 * p;
       const bool ok_n = mode == 0 && p < npairs_out && n < N;
       wsv[m][0] = ok_n ? __ldg(w_scale + n) : 0.f;
@@ -477,7 +498,8 @@ __global__ void __launch_bounds__(kDecGemmThreads, 2) decode_gemm_kernel(
         if (!ok && lane == 0) *reinterpret_cast<volatile int *>(abort_flag) = 1;
       }
       if (!ok) continue;
-      const int nkb = min(kDecKbStage, my_nk - si * kDecKbStage);
+      const int sj = si + rot < nstage ? si + rot : si + rot - nstage;
+      const int nkb = min(kDecKbStage, my_nk - sj * kDecKbStage);
       for (int kb = 0; kb < nkb; ++kb) {
         const uint8_t *wt = ring + slot * kDecStageBytes + kb * slab_w;
         const uint8_t *xt = ring + slot * kDecStageBytes + kDecWBytes + kb * kDecMaxM * 128;
@@ -513,24 +535,23 @@ __global__ void __launch_bounds__(kDecGemmThreads, 2) decode_gemm_kernel(
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int c = (ng * 4 + u) * 8 + 2 * tig;
-      *reinterpret_cast<int2 *>(P + ra * kDecRowsMax + c) = make_int2(acc[u][0], acc[u][1]);
-      *reinterpret_cast<int2 *>(P + rb * kDecRowsMax + c) = make_int2(acc[u][2], acc[u][3]);
+      *reinterpret_cast<int2 *>(P + ra * kDecPStride + c) = make_int2(acc[u][0], acc[u][1]);
+      *reinterpret_cast<int2 *>(P + rb * kDecPStride + c) = make_int2(acc[u][2], acc[u][3]);
     }
     cluster_sync();
-    // this CTA keeps channels [crank*half, (crank+1)*half) of the tile: token
-    // tok = tid/4, channel pairs p = tid%4 + 4m; its own partial plus the
-    // peer's, every load issued before the first add
+    // this CTA keeps channels [crank*half, (crank+1)*half) of the tile: its
+    // own partial plus the peer's, every load issued before the first add
     const uint32_t peer = crank ^ 1u;
     int2 own[4], oth[4];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-      const int p = (tid & 3) + 4 * m;
+      const int p = (tid >> 6) + 4 * m;
       own[m] = make_int2(0, 0);
       oth[m] = make_int2(0, 0);
       if (p < npairs_out) {
         const int c = static_cast<int>(crank) * half + 2 * p;
-        own[m] = *reinterpret_cast<const int2 *>(P + tok * kDecRowsMax + c);
-        oth[m] = ld_cluster_i2(map_to_rank(smem_u32(P + tok * kDecRowsMax + c), peer));
+        own[m] = *reinterpret_cast<const int2 *>(P + tok * kDecPStride + c);
+        oth[m] = ld_cluster_i2(map_to_rank(smem_u32(P + tok * kDecPStride + c), peer));
       }
     }
     int2 accv[4];
@@ -545,8 +566,7 @@ __global__ void __launch_bounds__(kDecGemmThreads, 2) decode_gemm_kernel(
     const bool any_lora = lora && mode != 1;
     if (any_lora) {
       asm volatile("griddepcontrol.wait;" ::: "memory");
-      int rmax = 0;
-      for (int t = 0; t < mt; ++t) rmax = max(rmax, ctl.tok_rank[t]);
+      const int rmax = ctl.rmax;
       for (int jb = 0; jb < rmax; jb += 16) {
         const int j = jb + (tid & 15);
         float pv[4][kDecShrinkSplitMax];
@@ -568,7 +588,7 @@ __global__ void __launch_bounds__(kDecGemmThreads, 2) decode_gemm_kernel(
             float sacc = 0.f;  // zero in the padding columns
 #pragma unroll
             for (int ks = 0; ks < kDecShrinkSplitMax; ++ks) sacc += pv[u][ks];
-            Tm[t * kDecMaxRank + j] = __fmul_rn(ctl.xs[t], sacc);
+            Tm[t * kDecTStride + j] = __fmul_rn(ctl.xs[t], sacc);
           }
         }
       }
@@ -582,12 +602,12 @@ __global__ void __launch_bounds__(kDecGemmThreads, 2) decode_gemm_kernel(
     const bool aborted = *abort_flag != 0;
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-      const int p = (tid & 3) + 4 * m;
+      const int p = (tid >> 6) + 4 * m;
       const int64_t n = c0 + 2 * p;
       if (p >= npairs_out || tok >= mt || n >= N || aborted) continue;
       float d0 = 0.f, d1 = 0.f;
       if (any_lora && r_i > 0) {
-        const float *Ti = Tm + tok * kDecMaxRank;
+        const float *Ti = Tm + tok * kDecTStride;
         for (int j = 0; j < r_i; j += 8) {
           const float4 t0 = *reinterpret_cast<const float4 *>(Ti + j);
           const float4 t1 = *reinterpret_cast<const float4 *>(Ti + j + 4);
