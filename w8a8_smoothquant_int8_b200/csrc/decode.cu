@@ -10,17 +10,17 @@
 //                       launch at once, so both stream side by side;
 //   kernel 2 (GEMM + expand), CTA pairs (thread-block clusters of two): each
 //                       pair owns a tile of up to 64 output channels and each
-//                       CTA of the pair one half of K, so a CTA streams its
-//                       half of the Wq tile and the matching half of Xq
-//                       through a TMA ring once; acc = Xq Wq^T with int8
-//                       tensor-core MMAs (m16n8k32, exact int32); the two
-//                       halves are added through distributed shared memory;
-//                       the B' rows of the CTA's output channels are
-//                       bulk-copied into shared memory while the weights
-//                       stream; after the shrink grid has completed
-//                       (programmatic dependent launch), T = x_scale * (sum of
-//                       the partials in a fixed order) and
-//                       Y = bf16(acc*xs*ws + T B_a^T).
+//                       CTA of the pair one half of K; the Wq tile streams in
+//                       through cp.async on the load/store path (a 2D TMA box
+//                       of short rows from HBM is issued too slowly to keep
+//                       an SM's share of the bandwidth) beside one TMA box of
+//                       Xq per stage, and acc = Xq Wq^T runs on the tensor
+//                       cores (tcgen05, exact int32 in tensor memory); the
+//                       pair adds its halves with one bulk copy from shared
+//                       memory to the peer's; after the shrink grid has
+//                       completed (programmatic dependent launch),
+//                       T = x_scale * (sum of the partials in a fixed order)
+//                       and Y = bf16(acc*xs*ws + T B_a^T).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -126,11 +126,11 @@ __device__ void decode_lookup(const int32_t *__restrict__ seg_offsets,
 // Thread t covers 8 consecutive K elements per pass and loads the 16 A' rows
 // of a rank group together (all of the block's 16 x 4 KB at once).
 // ---------------------------------------------------------------------------
-// At most 104 registers a thread: an SM's registers are split between its
+// At most 96 registers a thread: an SM's registers are split between its
 // four sub-partitions (16K each) and a block's warps are dealt to them in
-// turn, so a GEMM CTA (9 warps of 96 registers: 3 on one sub-partition) fits
-// beside a shrink block (2 warps on each) only while 3*96 + 2*r <= 512.
-__global__ void __maxnreg__(104) decode_shrink_kernel(
+// turn, so a GEMM CTA (12 warps of 96 registers: 3 on each sub-partition)
+// fits beside a shrink block (2 warps on each) only while 3*96 + 2*r <= 512.
+__global__ void __maxnreg__(96) decode_shrink_kernel(
     const int8_t *__restrict__ Xq, int64_t M, int64_t K, int ksplit,
     const uint16_t *__restrict__ A_pack, const int32_t *__restrict__ lora_offset,
     const int32_t *__restrict__ lora_rank, int n_adapters, int64_t R,
@@ -214,74 +214,97 @@ __global__ void __maxnreg__(104) decode_shrink_kernel(
 
 // ---------------------------------------------------------------------------
 // kernel 2: int8 GEMM + LoRA expand on CTA pairs.
-// A tile is `tile_units` groups of 8 output channels (at most 64 channels);
-// tiles are dealt to the pairs in turn.  Per CTA and tile:
-//   warp 8 (producer) streams the CTA's K half in stages of two 128-byte K
-//     blocks: one TMA copy of the tile's Wq rows and one of the 64 Xq rows,
-//     each a 3D box over the K blocks (two boxes per operand per stage when
-//     K is not a multiple of 128), lanes 0 and 1 issuing together.  A copy
-//     costs a few hundred ns to issue whatever its size, so the copies are
-//     made large.  Before its first tile it also bulk-copies the B' rows of
-//     the CTA's output channels when the tokens use at least half of the
-//     pack's columns;
-//   warps 0-7 (compute): warp w owns tokens [16(w&3), +16) and channel groups
-//     [4(w>>2), +4) of the tile; the K loop's int32 partials go to shared
-//     memory, the pair adds them through distributed shared memory (CTA c
-//     keeps channels [c*half, (c+1)*half) of the tile), then the epilogue.
-// Loads that the tail depends on (peer partials, the shrink's partial sums,
-// w_scale) are all issued before any of them is used.  Every spin-wait is
-// bounded; all threads of both CTAs pass the same barriers in the same order,
-// also after a wait that ran out.
+// A tile is `tile_units` groups of 8 output channels (at most 64); tiles are
+// dealt to the pairs in turn and each CTA of a pair takes one half of K.
+// Per CTA and tile:
+//   warps 3-11 (loaders) stream the CTA's K half in stages of two 128-byte K
+//     blocks: the tile's Wq rows by 16-byte cp.async copies (256 contiguous
+//     bytes of a row per stage, stored in the 128-byte swizzled layout the
+//     tensor core reads; a warp keeps only a few dozen copies in flight, so
+//     nine warps share them), and the 64 Xq rows by one TMA box of warp 11's
+//     lane 0 (every CTA reads the same Xq, so it comes from L2);
+//   warp 0, lane 0 issues the tensor-core MMAs of each stage as it lands:
+//     D[ch, tok] += Wq[ch, k] Xq[tok, k] with M = 128 channel rows (rows past
+//     the tile read bytes of the next slab; their results are never used),
+//     N = 64 tokens, exact int32 accumulators in tensor memory;
+//   warps 1-2 meanwhile find each token's adapter and, once the shrink grid
+//     has completed, form T = x_scale * (sum of the shrink's slices), each
+//     in one round of loads (a load issued while the SM streams waits behind
+//     the copies in flight; for ranks above 64 T is formed after the K loop
+//     where the stages were);
+//   then warps 0-1 move D to shared memory, the channels the peer finishes
+//     go to the peer in one bulk copy counted on its mbarrier, and warps 0-7
+//     finish the channels this CTA keeps, one channel per lane and 8 tokens
+//     per warp (their B' words requested before the peer's partials are
+//     awaited): acc = own + peer partial, delta = T B_a^T,
+//     Y = bf16(acc*xs*ws + delta).
+// Every wait on another thread is bounded; all threads of both CTAs pass the
+// same barriers in the same order, also after a wait that ran out, and no
+// CTA exits while a copy into its shared memory or a tensor-core operation
+// may still be in flight.
 // ---------------------------------------------------------------------------
 constexpr int kDecTileUnits = 8;                     // 8-channel groups per tile, at most
 constexpr int kDecRowsMax = 8 * kDecTileUnits;       // 64 output channels
 constexpr int kDecKbStage = 2;                       // 128-byte K blocks per stage
-constexpr int kDecStages = 4;
+constexpr int kDecStages = 5;
 constexpr int kDecWBytes = kDecKbStage * kDecRowsMax * 128;  // Wq slabs of a stage (16 KB)
 constexpr int kDecXBytes = kDecKbStage * kDecMaxM * 128;     // Xq slabs of a stage (16 KB)
 constexpr int kDecStageBytes = kDecWBytes + kDecXBytes;
-constexpr int kDecBBytes = (kDecRowsMax / 2) * SQ_MAX_LORA_COLS * 2;  // 64 KB
-constexpr int kDecComputeWarps = 8;
-constexpr int kDecComputeThreads = 32 * kDecComputeWarps;
-constexpr int kDecGemmThreads = kDecComputeThreads + 32;
-// named barriers: 1 compute warps; 2 all warps after the token lookup;
-// 3 all warps after a tile's K loop; 4 all warps after a tile's epilogue
-constexpr int kBarCompute = 1, kBarLookup = 2, kBarRingFree = 3, kBarTileEnd = 4;
+constexpr int kDecRingBytes = kDecStages * kDecStageBytes;
+constexpr int kDecKeepMax = kDecRowsMax / 2;                 // channels a CTA finishes
+constexpr int kDecTEarlyCols = 64;                           // T has its own region up to this rank
+constexpr int kDecTEarlyBytes = kDecMaxM * kDecTEarlyCols * 4;
+constexpr int kDecRecvBytes = kDecMaxM * kDecKeepMax * 4;    // the peer's partials
+constexpr int kDecEpiWarps = 8;
+constexpr int kDecEpiThreads = 32 * kDecEpiWarps;
+constexpr int kDecGemmThreads = kDecEpiThreads + 128;       // warps 8-11 only load
+constexpr int kDecLookupThreads = 64;                        // warps 1-2
+constexpr int kDecFirstLoader = 3;                           // warps 3-11 load Wq
+constexpr int kDecLoaderThreads = kDecGemmThreads - 32 * kDecFirstLoader;
+constexpr int kDecXWarp = kDecGemmThreads / 32 - 1;          // warp 11 also loads Xq
+constexpr uint32_t kDecTmemCols = 64;
+constexpr uint32_t kDecIdesc = idesc_i8_s32(128, kDecMaxM);
+// full barrier of a stage: one cp.async arrival per loader thread; the Xq
+// box of the stage is counted on a barrier of its own (xfull)
+// after the K loop the ring holds the partials sent to the peer [64][peer
+// channels], this CTA's own partials [64][32], T [64][rank padded to 16]
+// when it has no room of its own, and the epilogue's B' words: either the
+// kept channels' whole B' rows (row stride 2R + 16 bytes, so that lanes on
+// consecutive rows hit distinct banks) or 16 words of 16 bytes per thread,
+// stored [word][thread]
+constexpr int kDecSendOff = 0, kDecOwnOff = 8192, kDecTOff = 16384;
+constexpr int kDecBOff = kDecTOff + kDecMaxM * kDecMaxRank * 4;
+static_assert(kDecBOff + 16 * kDecEpiThreads * 16 <= kDecRingBytes, "T and B' must fit the ring");
+static_assert(kDecBOff + kDecKeepMax * (2 * SQ_MAX_LORA_COLS + 16) <= kDecRingBytes,
+              "the kept B' rows must fit the ring");
+// the MMA of K block 1 reads 128 rows from its slab: still inside the stage
+static_assert((kDecKbStage - 1) * kDecRowsMax * 128 + 128 * 128 <= kDecStageBytes,
+              "the channel rows an MMA reads must stay inside its stage");
+// named barriers: 1 warps 1-2 (token lookup); 2 warps 0-7; 3 all warps at a tile's end
+constexpr int kBarLookup = 1, kBarEpi = 2, kBarTileEnd = 3;
 
 struct DecodeCtl {
-  uint64_t full[kDecStages];
-  uint64_t empty[kDecStages];
-  uint64_t bfull;                  // B' rows landed
+  uint64_t full[kDecStages];       // Wq bytes of the stage landed
+  uint64_t xfull[kDecStages];      // Xq bytes of the stage landed
+  uint64_t empty[kDecStages];      // the stage's MMAs have read it
+  uint64_t accfull;                // the tile's MMAs have completed
+  uint64_t rbar;                   // the peer's partials have landed
+  uint64_t bbar;                   // the kept channels' B' rows have landed
+  uint32_t tmem_base;
   int tok_off[kDecMaxM];           // adapter column offset per token
   int tok_rank[kDecMaxM];          // adapter rank per token (0: none)
   float xs[kDecMaxM];              // x_scale per token
   DecodeTables tb;
   int abort;
-  int bdense;                      // B' rows staged in shared memory (first tile)
   int rmax;                        // largest rank among the tokens
+  int b_dense;                     // the tokens use at least half of the B' columns
+  int t_early;                     // T formed during the K loop, in its own region
 };
-// after the K loop the ring holds the int32 partials [64][64] and then T [64][256] fp32
-// (row strides padded so that the epilogue's lanes, which walk tokens, hit
-// distinct shared-memory banks)
-constexpr int kDecPStride = kDecRowsMax + 2;         // int32 per partial row
-constexpr int kDecTStride = kDecMaxRank + 4;         // fp32 per T row
-constexpr int kDecPartBytes = (kDecMaxM * kDecPStride * 4 + 15) / 16 * 16;
-static_assert(kDecPartBytes + kDecMaxM * kDecTStride * 4 <= kDecStages * kDecStageBytes,
-              "partials and T must fit the ring");
 
-constexpr size_t kDecSmemBytes =
-    static_cast<size_t>(kDecStages) * kDecStageBytes + kDecBBytes + sizeof(DecodeCtl) + 1024;
+constexpr size_t kDecSmemBytes = static_cast<size_t>(kDecRingBytes) + kDecRecvBytes +
+                                 kDecTEarlyBytes + sizeof(DecodeCtl) + 1024;
 
-__device__ __forceinline__ void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                             uint32_t b1) {
-  asm(
-      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 "
-      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// 8 bf16 (one 16-byte word) times 8 fp32 values, added to d
+// 8 bf16 (one 16-byte word) times 8 fp32 values, added to d in order
 __device__ __forceinline__ float dot8_bf16(const uint4 &w, const float4 &t0, const float4 &t1,
                                            float d) {
   d = fmaf(t0.x, __uint_as_float(w.x << 16), d);
@@ -295,11 +318,86 @@ __device__ __forceinline__ float dot8_bf16(const uint4 &w, const float4 &t0, con
   return d;
 }
 
-// (at most 112 registers a thread: a block of the shrink fits beside it on an SM)
-__global__ void __launch_bounds__(kDecGemmThreads, 2) decode_gemm_kernel(
-    const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-    int view3d, const float *__restrict__ x_scale, const float *__restrict__ w_scale, int64_t M,
-    int64_t N, int64_t K, int mode, const uint16_t *__restrict__ B_pack,
+// T[t][j] = x_scale[t] * (sum over the shrink's K slices, in order, of its
+// partial sums) for tokens t < mt and j < tstride (zero for j >= rank_t).
+// Work goes by quads of four consecutive j (tstride is a multiple of 16 and
+// a partial-sum row holds kDecMaxRank values, so a quad never leaves its
+// row; values past the rank are read but not used).  Each thread takes kB
+// quads at a time and loads two slices of each per round (one round when K
+// is at most two slices).
+template <int kB>
+__device__ void decode_form_t(float *T, int tstride, const float *part, int64_t M, int ksplit,
+                              int mt, const DecodeCtl &ctl, int tid, int nthr) {
+  const int qrow = tstride >> 2;
+  const int nq = mt * qrow;
+  for (int q0 = tid; q0 < nq; q0 += kB * nthr) {
+    float4 sacc[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) sacc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int ks0 = 0; ks0 < ksplit; ks0 += 2) {
+      float4 v[kB][2];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int qq = q0 + u * nthr;
+        const int t = qq < nq ? qq / qrow : 0, j = 4 * (qq - t * qrow);
+        const bool use = qq < nq && j < ctl.tok_rank[t];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          v[u][h] = (use && ks0 + h < ksplit)
+                        ? *reinterpret_cast<const float4 *>(
+                              part + (static_cast<int64_t>(ks0 + h) * M + t) * kDecMaxRank + j)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          sacc[u].x += v[u][h].x;
+          sacc[u].y += v[u][h].y;
+          sacc[u].z += v[u][h].z;
+          sacc[u].w += v[u][h].w;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int qq = q0 + u * nthr;
+      if (qq < nq) {
+        const int t = qq / qrow, j = 4 * (qq - t * qrow);
+        const int r = ctl.tok_rank[t];
+        const float xs = ctl.xs[t];
+        float4 o;
+        o.x = j + 0 < r ? __fmul_rn(xs, sacc[u].x) : 0.f;
+        o.y = j + 1 < r ? __fmul_rn(xs, sacc[u].y) : 0.f;
+        o.z = j + 2 < r ? __fmul_rn(xs, sacc[u].z) : 0.f;
+        o.w = j + 3 < r ? __fmul_rn(xs, sacc[u].w) : 0.f;
+        *reinterpret_cast<float4 *>(T + t * tstride + j) = o;
+      }
+    }
+  }
+}
+
+// B' words [jb, jb + 16) of channel row `brow` for the thread's tokens
+// tk0 .. tk0 + 7 into its slots of `bst` (slot 2u + h of token tk0 + u holds
+// columns jb + 8h .. jb + 8h + 7); words past a token's rank are not copied
+__device__ __forceinline__ void decode_stage_b(uint8_t *bst, int etid, const uint16_t *brow,
+                                               int tk0, int jb, int mt, const DecodeCtl &ctl) {
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int tok = tk0 + u;
+    const int r = tok < mt ? ctl.tok_rank[tok] : 0;
+    const uint16_t *bp = brow + (tok < mt ? ctl.tok_off[tok] : 0) + jb;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      if (jb + 8 * h < r) cp_async_16(bst + ((2 * u + h) * kDecEpiThreads + etid) * 16, bp + 8 * h);
+  }
+}
+
+// (at most 96 registers a thread: a block of the shrink fits beside it on an SM)
+__global__ void __maxnreg__(96) decode_gemm_kernel(
+    const __grid_constant__ CUtensorMap tm_x, int view3d, const int8_t *__restrict__ Wq,
+    const float *__restrict__ x_scale, const float *__restrict__ w_scale, int64_t M, int64_t N,
+    int64_t K, int mode, const uint16_t *__restrict__ B_pack,
     const int32_t *__restrict__ lora_offset, const int32_t *__restrict__ lora_rank,
     int n_adapters, int64_t R, const int32_t *__restrict__ seg_offsets,
     const int32_t *__restrict__ seg_adapter, int64_t S, const float *part, int ksplit,
@@ -307,16 +405,25 @@ __global__ void __launch_bounds__(kDecGemmThreads, 2) decode_gemm_kernel(
   extern __shared__ uint8_t dsm_raw[];
   uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
-  uint16_t *bsm = reinterpret_cast<uint16_t *>(ring + kDecStages * kDecStageBytes);
-  DecodeCtl &ctl = *reinterpret_cast<DecodeCtl *>(ring + kDecStages * kDecStageBytes + kDecBBytes);
-  int *P = reinterpret_cast<int *>(ring);                          // [64][kDecPStride] int32
-  float *Tm = reinterpret_cast<float *>(ring + kDecPartBytes);     // [64][kDecTStride] fp32
+  int *recv = reinterpret_cast<int *>(ring + kDecRingBytes);
+  float *t_own = reinterpret_cast<float *>(ring + kDecRingBytes + kDecRecvBytes);
+  DecodeCtl &ctl =
+      *reinterpret_cast<DecodeCtl *>(ring + kDecRingBytes + kDecRecvBytes + kDecTEarlyBytes);
+  int *sendp = reinterpret_cast<int *>(ring + kDecSendOff);
+  int *own = reinterpret_cast<int *>(ring + kDecOwnOff);
   volatile int *abort_flag = &ctl.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t crank = cluster_ctarank();
+  const uint32_t crank = cluster_ctarank(), peer = crank ^ 1u;
   const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
-  const bool lora = (part != nullptr);
-  const int tile_rows = 8 * tile_units, half = 4 * tile_units;
+  const bool lora = (part != nullptr) && mode != 1;
+  const int tile_rows = 8 * tile_units;
+  // channels [keep_lo, keep_lo + keep_cols) of a tile are finished here, the
+  // others by the peer
+  const int lo_units = (tile_units + 1) / 2;
+  const int keep_lo = crank == 0 ? 0 : 8 * lo_units;
+  const int keep_cols = crank == 0 ? 8 * lo_units : 8 * (tile_units - lo_units);
+  const int peer_lo = crank == 0 ? 8 * lo_units : 0;
+  const int peer_cols = tile_rows - keep_cols;
   const int slab_w = tile_rows * 128;  // bytes of one K block of the Wq tile
   const int nk = (mode == 2) ? 0 : static_cast<int>((K + 127) / 128);
   const int nk_half = (nk + 1) / 2;
@@ -330,314 +437,385 @@ __global__ void __launch_bounds__(kDecGemmThreads, 2) decode_gemm_kernel(
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) {
-      mbar_init(&ctl.full[s], 1);
-      mbar_init(&ctl.empty[s], kDecComputeWarps);
+      mbar_init(&ctl.full[s], kDecLoaderThreads);
+      mbar_init(&ctl.xfull[s], 1);
+      mbar_init(&ctl.empty[s], 1);
     }
-    mbar_init(&ctl.bfull, 1);
+    mbar_init(&ctl.accfull, 1);
+    mbar_init(&ctl.rbar, 1);
+    mbar_init(&ctl.bbar, 1);
     ctl.abort = 0;
-    ctl.bdense = 0;
+    ctl.rmax = 0;
+    ctl.b_dense = 0;
+    ctl.t_early = 0;
     fence_mbar_init();
   }
+  if (warp == 0) {
+    tmem_alloc(&ctl.tmem_base, kDecTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem_base;
+  // the peer pushes its partials only after this arrival: the receive
+  // barrier exists by then
+  cluster_arrive();
 
-  if (warp == kDecComputeWarps) {
-    // ---------------------------------------------------------- producer
-    if (lane == 0) {
-      prefetch_tmap(&tm_w);
-      prefetch_tmap(&tm_x);
-    }
-    int q = 0;  // stages issued so far (all tiles)
-    bool looked_up = false, b_issued = false, stop = false;
-    auto after_lookup = [&](int first_tile) {
-      // B' rows of this CTA's channels in the first tile, when the tokens use
-      // at least half of the pack's columns (else the epilogue reads the used
-      // columns from global memory)
-      group_bar(kBarLookup, kDecGemmThreads);
-      looked_up = true;
-      if (!lora || first_tile >= tiles || lane != 0 || R <= 0) return;
-      unsigned long long used = 0;  // 16-column groups (R <= 1024)
-      for (int i = 0; i < mt; ++i) {
-        const int r = ctl.tok_rank[i];
-        if (r > 0) {
-          const int g0 = ctl.tok_off[i] >> 4, g1 = (ctl.tok_off[i] + r + 15) >> 4;
-          for (int g = g0; g < g1; ++g) used |= 1ull << g;
-        }
-      }
-      if (2 * 16 * __popcll(used) < R) return;
-      const int64_t c0 = static_cast<int64_t>(first_tile) * tile_rows + crank * half;
-      const int64_t rows = max(static_cast<int64_t>(0), min(static_cast<int64_t>(half), N - c0));
-      if (rows <= 0) return;
-      const uint32_t bytes = static_cast<uint32_t>(rows * R * 2);
-      ctl.bdense = 1;
-      mbar_arrive_expect_tx(&ctl.bfull, bytes);
-      bulk_load(bsm, B_pack + c0 * R, bytes, &ctl.bfull);
-      b_issued = true;
-    };
-    for (int tile = pair; tile < tiles; tile += npairs) {
-      const int32_t n0 = tile * tile_rows;
-      for (int si = 0; si < nstage; ++si) {
-        const int slot = q % kDecStages;
-        const uint32_t ph = static_cast<uint32_t>(q / kDecStages) & 1u;
-        const int sj = si + rot < nstage ? si + rot : si + rot - nstage;
-        const int kbs = kb0 + sj * kDecKbStage;                       // first K block
-        const int nkb = min(kDecKbStage, kb0 + my_nk - kbs);          // this CTA's blocks
-        const int boxes = view3d ? kDecKbStage : nkb;                 // K blocks copied
-        bool got = true;
-        if (lane == 0 && !stop) {
-          // nothing more is issued once any wait has run out: a slot whose
-          // copy nobody waited for may still be written to
-          got = !*abort_flag && mbar_wait(&ctl.empty[slot], ph ^ 1u, timeout_ns, abort_flag) &&
-                !*abort_flag;
-          if (got)
-            mbar_arrive_expect_tx(&ctl.full[slot],
-                                  static_cast<uint32_t>(boxes * (slab_w + kDecMaxM * 128)));
-        }
-        got = __shfl_sync(0xffffffffu, got && !stop, 0);
-        if (!got) {
-          if (lane == 0 && !stop) {
-            *reinterpret_cast<volatile int *>(abort_flag) = 1;
-            record_device_error(SQ_ERR_DEVICE_TIMEOUT);
-          }
-          stop = true;
-        } else {
-          uint8_t *st = ring + slot * kDecStageBytes;
-          if (view3d) {
-            if (lane == 0) tma_load_3d(st, &tm_w, &ctl.full[slot], 0, n0, kbs);
-            if (lane == 1) tma_load_3d(st + kDecWBytes, &tm_x, &ctl.full[slot], 0, 0, kbs);
-          } else if (lane < 2 * nkb) {
-            const int kb = lane >> 1;
-            if ((lane & 1) == 0)
-              tma_load_2d(st + kb * slab_w, &tm_w, &ctl.full[slot], (kbs + kb) * 128, n0);
-            else
-              tma_load_2d(st + kDecWBytes + kb * kDecMaxM * 128, &tm_x, &ctl.full[slot],
-                          (kbs + kb) * 128, 0);
-          }
-          ++q;
-        }
-        if (!looked_up && (q == kDecStages || si == nstage - 1)) after_lookup(pair);
-      }
-      if (!looked_up) after_lookup(pair);
-      // every copy of this tile must land before the ring is reused (also
-      // after a wait that ran out: wait for the last use of each slot)
+  // ---------------------------------------------------------- loaders
+  // (warps 3-7 then join the epilogue; warps 8-11 only load)
+  int q = 0;  // stages issued so far by this warp (all tiles)
+  bool stop = false;
+  auto load_tile = [&](int64_t n0) {
+    const int ltid = static_cast<int>(threadIdx.x) - 32 * kDecFirstLoader;
+    const int rows = static_cast<int>(min(static_cast<int64_t>(tile_rows), N - n0));
+    const int8_t *wtile = Wq + n0 * K;
+    for (int si = 0; si < nstage && !stop; ++si) {
+      const int slot = q % kDecStages;
+      const uint32_t ph = static_cast<uint32_t>(q / kDecStages) & 1u;
+      const int sj = si + rot < nstage ? si + rot : si + rot - nstage;
+      const int kbs = kb0 + sj * kDecKbStage;               // first K block
+      const int nkb = min(kDecKbStage, kb0 + my_nk - kbs);  // this CTA's blocks
+      bool got = false;
       if (lane == 0) {
-        volatile int never = 0;
-        const int issued = q;
-        for (int k = 0; k < kDecStages && k < issued; ++k) {
-          const int last = issued - 1 - ((issued - 1 - k) % kDecStages);
-          mbar_wait(&ctl.full[last % kDecStages], static_cast<uint32_t>(last / kDecStages) & 1u,
-                    1000000000ull, &never);
+        // nothing more is issued once any wait has run out: a slot whose
+        // copy nobody waited for may still be written to
+        got = !*abort_flag && mbar_wait(&ctl.empty[slot], ph ^ 1u, timeout_ns, abort_flag) &&
+              !*abort_flag;
+        if (!got) {
+          *reinterpret_cast<volatile int *>(abort_flag) = 1;
+          record_device_error(SQ_ERR_DEVICE_TIMEOUT);
         }
       }
-      __syncwarp();
-      group_bar(kBarRingFree, kDecGemmThreads);
-      cluster_sync();  // partials written by both CTAs
-      cluster_sync();  // partials read by both CTAs
-      group_bar(kBarTileEnd, kDecGemmThreads);
+      if (!__shfl_sync(0xffffffffu, got, 0)) {
+        stop = true;
+        break;
+      }
+      uint8_t *st = ring + slot * kDecStageBytes;
+      // Wq: rows x nkb K blocks x 8 chunks of 16 bytes; consecutive threads
+      // take consecutive chunks of a row.  Chunks past K are not copied (the
+      // Xq box is zero there).
+      const int cshift = nkb == 2 ? 4 : 3;
+      const int total = rows << cshift;
+      const int8_t *src0 = wtile + static_cast<int64_t>(kbs) * 128;
+      const int64_t kleft = K - static_cast<int64_t>(kbs) * 128;  // bytes of K from kbs on
+      for (int idx = ltid; idx < total; idx += kDecLoaderThreads) {
+        const int row = idx >> cshift, cc = idx & ((1 << cshift) - 1);
+        if (cc * 16 < kleft) {
+          const int kb = cc >> 3, c = cc & 7;
+          cp_async_16(st + kb * slab_w + row * 128 + ((c ^ (row & 7)) << 4),
+                      src0 + static_cast<int64_t>(row) * K + cc * 16);
+        }
+      }
+      cp_async_mbar_arrive_noinc(&ctl.full[slot]);
+      if (warp == kDecXWarp && lane == 0) {
+        if (view3d) {
+          mbar_arrive_expect_tx(&ctl.xfull[slot], static_cast<uint32_t>(kDecXBytes));
+          tma_load_3d(st + kDecWBytes, &tm_x, &ctl.xfull[slot], 0, 0, kbs);
+        } else {
+          mbar_arrive_expect_tx(&ctl.xfull[slot], static_cast<uint32_t>(nkb * kDecMaxM * 128));
+          for (int kb = 0; kb < nkb; ++kb)
+            tma_load_2d(st + kDecWBytes + kb * kDecMaxM * 128, &tm_x, &ctl.xfull[slot],
+                        (kbs + kb) * 128, 0);
+        }
+      }
+      ++q;
     }
-    if (!looked_up) after_lookup(pair);
-    if (lane == 0 && b_issued) {
+  };
+  // every copy into shared memory has landed before the CTA exits (also
+  // after a wait that ran out: cp.async by each thread, the Xq boxes by the
+  // last use of each slot's barrier)
+  auto drain_loads = [&]() {
+    cp_async_wait_all();
+    if (warp == kDecXWarp && lane == 0) {
       volatile int never = 0;
-      mbar_wait(&ctl.bfull, 0, 1000000000ull, &never);
+      for (int k = 0; k < kDecStages && k < q; ++k) {
+        const int last = q - 1 - ((q - 1 - k) % kDecStages);
+        mbar_wait(&ctl.xfull[last % kDecStages], static_cast<uint32_t>(last / kDecStages) & 1u,
+                  1000000000ull, &never);
+      }
     }
+    __syncwarp();
+  };
+  if (warp >= kDecEpiWarps) {
+    if (warp == kDecXWarp && lane == 0) prefetch_tmap(&tm_x);
+    for (int tile = pair; tile < tiles; tile += npairs) {
+      load_tile(static_cast<int64_t>(tile) * tile_rows);
+      // the ring is reused for this tile's partials: the next tile's copies
+      // start after its epilogue
+      cluster_wait();
+      group_bar(kBarTileEnd, kDecGemmThreads);
+      cluster_arrive();
+    }
+    drain_loads();
+    cluster_wait();
     return;
   }
 
-  // ----------------------------------------------------------- compute
-  const int tid = threadIdx.x;
-  const int g = lane >> 2, tig = lane & 3;
-  if (lora)
-    decode_lookup(seg_offsets, seg_adapter, S, lora_offset, lora_rank, n_adapters, R, 0, mt, tid,
-                  kDecComputeThreads, kBarCompute, ctl.tb, ctl.tok_off, ctl.tok_rank);
-  else
-    for (int i = tid; i < kDecMaxM; i += kDecComputeThreads) ctl.tok_rank[i] = 0;
-  for (int i = tid; i < kDecMaxM; i += kDecComputeThreads)
-    ctl.xs[i] = (mode != 1 && i < M) ? __ldg(x_scale + i) : 0.f;
-  if (warp == 0) {  // (the lookup ended with a barrier of the compute warps)
-    int r = max(lane < mt ? ctl.tok_rank[lane] : 0, lane + 32 < mt ? ctl.tok_rank[lane + 32] : 0);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) r = max(r, __shfl_xor_sync(0xffffffffu, r, o));
-    if (lane == 0) ctl.rmax = r;
-  }
-  group_bar(kBarLookup, kDecGemmThreads);
-
-  const int mtile = warp & 3, ng = warp >> 2;
-  const int ra = mtile * 16 + g, rb = ra + 8;  // token rows of this lane's A fragments
-  int q = 0;
-  bool first = true;
-  for (int tile = pair; tile < tiles; tile += npairs) {
+  // ------------------------------------------------ MMA, lookup, epilogue
+  // B' rows of a tile's kept channels into L2 ahead of the epilogue, when the
+  // tokens read most of each row
+  auto prefetch_b = [&](int64_t n0) {
+    const int64_t c0 = n0 + keep_lo;
+    const int64_t rows =
+        max(static_cast<int64_t>(0), min(static_cast<int64_t>(keep_cols), N - c0));
+    if (ctl.b_dense && rows > 0)
+      bulk_prefetch_l2(B_pack + c0 * R, static_cast<uint32_t>(rows * R * 2));
+  };
+  const int etid = threadIdx.x;  // 0..255
+  int mq = 0;                    // stages consumed by the MMA thread (all tiles)
+  bool mma_ok = true;
+  int it = 0;
+  for (int tile = pair; tile < tiles; tile += npairs, ++it) {
     const int64_t n0 = static_cast<int64_t>(tile) * tile_rows;
-    const int64_t c0 = n0 + static_cast<int64_t>(crank) * half;  // this CTA's first channel
-    // epilogue: token tok = tid % 64 and channel pairs p = tid/64 + 4m of this
-    // CTA's half of the tile (a warp's lanes walk 32 tokens)
-    const int tok = tid & 63;
-    const int npairs_out = half / 2;
-    // w_scale of this thread's epilogue channels, loaded ahead of every wait
-    float wsv[4][2];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int p = (tid >> 6) + 4 * m;
-      const int64_t n = c0 + 2 * p;
-      const bool ok_n = mode == 0 && p < npairs_out && n < N;
-      wsv[m][0] = ok_n ? __ldg(w_scale + n) : 0.f;
-      wsv[m][1] = ok_n ? __ldg(w_scale + n + 1) : 0.f;
-    }
-    int acc[4][4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[u][e] = 0;
-    bool ok = true;
-    for (int si = 0; si < nstage; ++si, ++q) {
-      const int slot = q % kDecStages;
-      const uint32_t ph = static_cast<uint32_t>(q / kDecStages) & 1u;
-      // the warp leaves together: the mma.sync below needs all lanes.  A warp
-      // whose wait ran out raises the abort flag at once and hands no more
-      // stages back (the producer then issues nothing more)
-      if (ok) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&ctl.full[slot], ph, timeout_ns, abort_flag));
-        if (!ok && lane == 0) *reinterpret_cast<volatile int *>(abort_flag) = 1;
-      }
-      if (!ok) continue;
-      const int sj = si + rot < nstage ? si + rot : si + rot - nstage;
-      const int nkb = min(kDecKbStage, my_nk - sj * kDecKbStage);
-      for (int kb = 0; kb < nkb; ++kb) {
-        const uint8_t *wt = ring + slot * kDecStageBytes + kb * slab_w;
-        const uint8_t *xt = ring + slot * kDecStageBytes + kDecWBytes + kb * kDecMaxM * 128;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          // 16 contiguous K bytes (chunk 4h + tig of the 128-byte row, stored
-          // 128B-swizzled) of each operand row; the K order inside the 64
-          // bytes is a permutation that A and B share
-          const uint4 xa = *reinterpret_cast<const uint4 *>(xt + ra * 128 + (((4 * h + tig) ^ (ra & 7)) * 16));
-          const uint4 xb = *reinterpret_cast<const uint4 *>(xt + rb * 128 + (((4 * h + tig) ^ (rb & 7)) * 16));
-          const uint32_t fa0[4] = {xa.x, xb.x, xa.y, xb.y};
-          const uint32_t fa1[4] = {xa.z, xb.z, xa.w, xb.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            if (ng * 4 + u >= tile_units) continue;  // warp-uniform
-            const int row = (ng * 4 + u) * 8 + g;
-            const uint4 bw = *reinterpret_cast<const uint4 *>(wt + row * 128 + (((4 * h + tig) ^ (row & 7)) * 16));
-            mma_s8_16832(acc[u], fa0, bw.x, bw.y);
-            mma_s8_16832(acc[u], fa1, bw.z, bw.w);
+    // this thread's epilogue channel; its w_scale is loaded long before use
+    const int64_t n = n0 + keep_lo + lane;
+    const float ws_n = (mode == 0 && lane < keep_cols && n < N) ? __ldg(w_scale + n) : 0.f;
+    if (warp == 0) {
+      if (lane == 0) {
+        bool any = false;
+        for (int si = 0; si < nstage; ++si, ++mq) {
+          const int slot = mq % kDecStages;
+          const uint32_t ph = static_cast<uint32_t>(mq / kDecStages) & 1u;
+          if (mma_ok) {
+            mma_ok = mbar_wait(&ctl.full[slot], ph, timeout_ns, abort_flag) &&
+                     mbar_wait(&ctl.xfull[slot], ph, timeout_ns, abort_flag);
+            if (!mma_ok) {
+              *reinterpret_cast<volatile int *>(abort_flag) = 1;
+              record_device_error(SQ_ERR_DEVICE_TIMEOUT);
+            }
           }
+          if (!mma_ok) continue;
+          // the Wq bytes were written by cp.async (generic proxy)
+          fence_proxy_async_shared();
+          tc_fence_after();
+          const int sj = si + rot < nstage ? si + rot : si + rot - nstage;
+          const int nkb = min(kDecKbStage, my_nk - sj * kDecKbStage);
+          const uint32_t wa = smem_u32(ring + slot * kDecStageBytes);
+          const uint32_t xa = wa + kDecWBytes;
+          for (int kb = 0; kb < nkb; ++kb) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              mma_i8(tmem, sdesc_kmajor_sw128(wa + kb * slab_w + 32 * k),
+                     sdesc_kmajor_sw128(xa + kb * kDecMaxM * 128 + 32 * k), kDecIdesc,
+                     any ? 1u : 0u);
+              any = true;
+            }
+          }
+          mma_commit(&ctl.empty[slot]);
         }
+        if (any)
+          mma_commit(&ctl.accfull);
+        else
+          mbar_arrive(&ctl.accfull);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl.empty[slot]);
-    }
-    if (!ok) {
-      *reinterpret_cast<volatile int *>(abort_flag) = 1;
-      record_device_error(SQ_ERR_DEVICE_TIMEOUT);
-    }
-    // every copy into the ring has landed (the producer waited): the
-    // partials go where the stages were
-    group_bar(kBarRingFree, kDecGemmThreads);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int c = (ng * 4 + u) * 8 + 2 * tig;
-      *reinterpret_cast<int2 *>(P + ra * kDecPStride + c) = make_int2(acc[u][0], acc[u][1]);
-      *reinterpret_cast<int2 *>(P + rb * kDecPStride + c) = make_int2(acc[u][2], acc[u][3]);
-    }
-    cluster_sync();
-    // this CTA keeps channels [crank*half, (crank+1)*half) of the tile: its
-    // own partial plus the peer's, every load issued before the first add
-    const uint32_t peer = crank ^ 1u;
-    int2 own[4], oth[4];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int p = (tid >> 6) + 4 * m;
-      own[m] = make_int2(0, 0);
-      oth[m] = make_int2(0, 0);
-      if (p < npairs_out) {
-        const int c = static_cast<int>(crank) * half + 2 * p;
-        own[m] = *reinterpret_cast<const int2 *>(P + tok * kDecPStride + c);
-        oth[m] = ld_cluster_i2(map_to_rank(smem_u32(P + tok * kDecPStride + c), peer));
-      }
-    }
-    int2 accv[4];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) accv[m] = make_int2(own[m].x + oth[m].x, own[m].y + oth[m].y);
-    cluster_sync();
-    // ---- LoRA: T = x_scale * (sum of the shrink's slices in order), after
-    //      the shrink grid has completed; each thread takes four (token, rank)
-    //      entries of a 16-rank group and loads all their slices at once
-    const int r_i = (tok < mt) ? ctl.tok_rank[tok] : 0;
-    const int off_i = (tok < mt) ? ctl.tok_off[tok] : 0;
-    const bool any_lora = lora && mode != 1;
-    if (any_lora) {
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      const int rmax = ctl.rmax;
-      for (int jb = 0; jb < rmax; jb += 16) {
-        const int j = jb + (tid & 15);
-        float pv[4][kDecShrinkSplitMax];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int t = (tid >> 4) + 16 * u;
-          const int r = (t < mt) ? ctl.tok_rank[t] : 0;
-#pragma unroll
-          for (int ks = 0; ks < kDecShrinkSplitMax; ++ks)
-            pv[u][ks] = (j < r && ks < ksplit)
-                            ? part[(static_cast<int64_t>(ks) * M + t) * kDecMaxRank + j]
-                            : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int t = (tid >> 4) + 16 * u;
-          const int r = (t < mt) ? ctl.tok_rank[t] : 0;
-          if (t < mt && j < ((r + 15) & ~15)) {
-            float sacc = 0.f;  // zero in the padding columns
-#pragma unroll
-            for (int ks = 0; ks < kDecShrinkSplitMax; ++ks) sacc += pv[u][ks];
-            Tm[t * kDecTStride + j] = __fmul_rn(ctl.xs[t], sacc);
-          }
-        }
-      }
-      group_bar(kBarCompute, kDecComputeThreads);
-    }
-    const bool use_bsm = first && ctl.bdense;
-    if (use_bsm && !mbar_wait(&ctl.bfull, 0, timeout_ns, abort_flag)) {
-      *reinterpret_cast<volatile int *>(abort_flag) = 1;
-      record_device_error(SQ_ERR_DEVICE_TIMEOUT);
-    }
-    const bool aborted = *abort_flag != 0;
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int p = (tid >> 6) + 4 * m;
-      const int64_t n = c0 + 2 * p;
-      if (p >= npairs_out || tok >= mt || n >= N || aborted) continue;
-      float d0 = 0.f, d1 = 0.f;
-      if (any_lora && r_i > 0) {
-        const float *Ti = Tm + tok * kDecTStride;
-        for (int j = 0; j < r_i; j += 8) {
-          const float4 t0 = *reinterpret_cast<const float4 *>(Ti + j);
-          const float4 t1 = *reinterpret_cast<const float4 *>(Ti + j + 4);
-          uint4 w0, w1;
-          if (use_bsm) {
-            w0 = *reinterpret_cast<const uint4 *>(bsm + (n - c0) * R + off_i + j);
-            w1 = *reinterpret_cast<const uint4 *>(bsm + (n + 1 - c0) * R + off_i + j);
-          } else {
-            w0 = __ldg(reinterpret_cast<const uint4 *>(B_pack + n * R + off_i + j));
-            w1 = __ldg(reinterpret_cast<const uint4 *>(B_pack + (n + 1) * R + off_i + j));
-          }
-          d0 = dot8_bf16(w0, t0, t1, d0);
-          d1 = dot8_bf16(w1, t0, t1, d1);
-        }
-      }
-      if (mode == 0) {
-        const float xs = ctl.xs[tok];
-        const float y0 = __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(accv[m].x), xs), wsv[m][0]), d0);
-        const float y1 = __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(accv[m].y), xs), wsv[m][1]), d1);
-        __nv_bfloat162 hh = __floats2bfloat162_rn(y0, y1);
-        *reinterpret_cast<uint32_t *>(static_cast<uint16_t *>(out) + tok * N + n) =
-            *reinterpret_cast<uint32_t *>(&hh);
-      } else if (mode == 1) {
-        *reinterpret_cast<int2 *>(static_cast<int32_t *>(out) + tok * N + n) = accv[m];
+    } else if (warp >= kDecFirstLoader) {
+      load_tile(n0);
+    } else if (it == 0) {
+      // token lookup and x_scale in one round of loads, then the largest rank
+      // and whether the tokens read most of the B' columns
+      const int ltid = etid - 32;
+      static_assert(kDecMaxM == kDecLookupThreads, "one token a lookup thread");
+      const float xsv = (mode != 1 && ltid < M) ? __ldg(x_scale + ltid) : 0.f;
+      if (lora) {
+        decode_lookup(seg_offsets, seg_adapter, S, lora_offset, lora_rank, n_adapters, R, 0, mt,
+                      ltid, kDecLookupThreads, kBarLookup, ctl.tb, ctl.tok_off, ctl.tok_rank);
       } else {
-        *reinterpret_cast<float2 *>(static_cast<float *>(out) + tok * N + n) = make_float2(d0, d1);
+        ctl.tok_rank[ltid] = 0;
+        ctl.tok_off[ltid] = 0;
+      }
+      ctl.xs[ltid] = xsv;
+      group_bar(kBarLookup, kDecLookupThreads);
+      if (warp == 1) {
+        // lane l takes tokens l and l + 32; 16-column groups of the pack the
+        // tokens use (R <= 1024)
+        int r = 0;
+        uint32_t used_lo = 0, used_hi = 0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int i = lane + 32 * h;
+          const int ri = i < mt ? ctl.tok_rank[i] : 0;
+          r = max(r, ri);
+          if (ri > 0) {
+            const int g0 = ctl.tok_off[i] >> 4, g1 = (ctl.tok_off[i] + ri + 15) >> 4;
+            for (int g = g0; g < g1; ++g) {
+              if (g < 32)
+                used_lo |= 1u << g;
+              else
+                used_hi |= 1u << (g - 32);
+            }
+          }
+        }
+        r = __reduce_max_sync(0xffffffffu, r);
+        used_lo = __reduce_or_sync(0xffffffffu, used_lo);
+        used_hi = __reduce_or_sync(0xffffffffu, used_hi);
+        if (lane == 0) {
+          ctl.rmax = r;
+          ctl.b_dense = lora && r > 0 && 2 * 16 * (__popc(used_lo) + __popc(used_hi)) >= R;
+          ctl.t_early = ((r + 15) & ~15) <= kDecTEarlyCols;
+          prefetch_b(n0);
+        }
+      }
+      group_bar(kBarLookup, kDecLookupThreads);
+      if (lora && ctl.rmax > 0 && ctl.t_early) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        decode_form_t<4>(t_own, (ctl.rmax + 15) & ~15, part, M, ksplit, mt, ctl, ltid,
+                          kDecLookupThreads);
       }
     }
-    first = false;
+    if (warp == 1 && lane == 0 && it > 0) prefetch_b(n0);
+    group_bar(kBarEpi, kDecEpiThreads);
+    const int rmax = ctl.rmax;
+    const int tstride = (rmax + 15) & ~15;
+    // ---- D -> shared memory (warps 0-1, thread = channel 32*warp + lane)
+    if (warp < 2) {
+      const bool acc_ok =
+          __all_sync(0xffffffffu, mbar_wait(&ctl.accfull, static_cast<uint32_t>(it) & 1u,
+                                             timeout_ns, abort_flag));
+      if (!acc_ok && lane == 0) {
+        *reinterpret_cast<volatile int *>(abort_flag) = 1;
+        record_device_error(SQ_ERR_DEVICE_TIMEOUT);
+      }
+      tc_fence_after();
+      const bool have = acc_ok && my_nk > 0;  // warp-uniform
+      const int c = 32 * warp + lane;
+      const bool mine = c >= keep_lo && c < keep_lo + keep_cols;
+      int *dst = mine ? own + (c - keep_lo) : sendp + (c - peer_lo);
+      const int stride = mine ? kDecKeepMax : peer_cols;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[32];
+        if (have) {
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32 * h, v);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) v[t] = 0;
+        }
+        if (c < tile_rows) {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) dst[(32 * h + t) * stride] = static_cast<int>(v[t]);
+        }
+      }
+      // the send buffer is read by the bulk copy (async proxy)
+      fence_proxy_async_shared();
+    }
+    // the peer has finished with its receive buffer (previous tile)
+    cluster_wait();
+    group_bar(kBarEpi, kDecEpiThreads);
+    if (etid == 0 && peer_cols > 0) {
+      bulk_copy_to_cta(map_to_rank(smem_u32(recv), peer), sendp,
+                       static_cast<uint32_t>(kDecMaxM * peer_cols * 4),
+                       map_to_rank(smem_u32(&ctl.rbar), peer));
+      bulk_commit_group();
+    }
+    if (etid == 32) mbar_arrive_expect_tx(&ctl.rbar, static_cast<uint32_t>(kDecMaxM * keep_cols * 4));
+    // ---- epilogue: channel keep_lo + lane, tokens [8*warp, 8*warp + 8)
+    const bool live = lane < keep_cols && n < N;
+    const uint16_t *brow = B_pack + (live ? n : 0) * R;
+    float *T = t_own;
+    if (lora && rmax > 0 && !ctl.t_early) {
+      // T had no room of its own: it goes where the stages were
+      T = reinterpret_cast<float *>(ring + kDecTOff);
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      decode_form_t<2>(T, tstride, part, M, ksplit, mt, ctl, etid, kDecEpiThreads);
+      group_bar(kBarEpi, kDecEpiThreads);
+    }
+    // the B' words go out before the peer's partials are awaited: whole
+    // rows by bulk copies when the tokens read most of them, else each
+    // thread's words by cp.async
+    uint8_t *bst = ring + kDecBOff;
+    const bool b_rows = lora && ctl.b_dense;
+    const uint32_t brow_stride = static_cast<uint32_t>(R * 2 + 16);
+    const int b_nrows =
+        static_cast<int>(max(static_cast<int64_t>(0),
+                             min(static_cast<int64_t>(keep_cols), N - (n0 + keep_lo))));
+    if (b_rows && etid == 0 && b_nrows > 0) {
+      mbar_arrive_expect_tx(&ctl.bbar, static_cast<uint32_t>(b_nrows * R * 2));
+      for (int i = 0; i < b_nrows; ++i)
+        bulk_load(bst + i * brow_stride, B_pack + (n0 + keep_lo + i) * R,
+                  static_cast<uint32_t>(R * 2), &ctl.bbar);
+    }
+    const bool b_staged = lora && !b_rows && rmax <= 16;
+    if (live && b_staged) decode_stage_b(bst, etid, brow, 8 * warp, 0, mt, ctl);
+    if (!mbar_wait(&ctl.rbar, static_cast<uint32_t>(it) & 1u, timeout_ns, abort_flag)) {
+      *reinterpret_cast<volatile int *>(abort_flag) = 1;
+      record_device_error(SQ_ERR_DEVICE_TIMEOUT);
+    }
+    if (b_rows && b_nrows > 0 &&
+        !mbar_wait(&ctl.bbar, static_cast<uint32_t>(it) & 1u, timeout_ns, abort_flag)) {
+      *reinterpret_cast<volatile int *>(abort_flag) = 1;
+      record_device_error(SQ_ERR_DEVICE_TIMEOUT);
+    }
+    if (b_staged) cp_async_wait_all();
+    // one rolled loop over the thread's tokens: the epilogue runs once per
+    // CTA, so its code is fetched cold and is kept short
+    if (live && *abort_flag == 0) {
+      const uint8_t *mine_row = bst + lane * brow_stride;
+#pragma unroll 1
+      for (int u = 0; u < 8; ++u) {
+        const int tok = 8 * warp + u;
+        if (tok >= mt) break;
+        const int r = lora ? ctl.tok_rank[tok] : 0;
+        const int off = ctl.tok_off[tok];
+        float d = 0.f;
+#pragma unroll 1
+        for (int j = 0; j < r; j += 8) {
+          // the 8 B' words [j, j + 8): from the kept rows, this thread's
+          // staged words, or (a sparse pack with ranks above 16) global memory
+          uint4 w;
+          if (b_rows)
+            w = *reinterpret_cast<const uint4 *>(mine_row + (off + j) * 2);
+          else if (b_staged)
+            w = *reinterpret_cast<const uint4 *>(
+                bst + ((2 * u + (j >> 3)) * kDecEpiThreads + etid) * 16);
+          else
+            w = __ldg(reinterpret_cast<const uint4 *>(brow + off + j));
+          const float *Ti = T + tok * tstride + j;
+          d = dot8_bf16(w, *reinterpret_cast<const float4 *>(Ti),
+                        *reinterpret_cast<const float4 *>(Ti + 4), d);
+        }
+        const int acc = own[tok * kDecKeepMax + lane] + recv[tok * keep_cols + lane];
+        if (mode == 0) {
+          const float y =
+              __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(acc), ctl.xs[tok]), ws_n), d);
+          static_cast<__nv_bfloat16 *>(out)[tok * N + n] = __float2bfloat16_rn(y);
+        } else if (mode == 1) {
+          static_cast<int32_t *>(out)[tok * N + n] = acc;
+        } else {
+          static_cast<float *>(out)[tok * N + n] = d;
+        }
+      }
+    }
+    // (copies issued by a thread that then skipped the epilogue)
+    cp_async_wait_all();
+    // the send buffer has been read before the ring is reused
+    if (etid == 0 && peer_cols > 0) bulk_wait_group_read<0>();
+    tc_fence_before();
     group_bar(kBarTileEnd, kDecGemmThreads);
+    cluster_arrive();
+  }
+  if (warp >= kDecFirstLoader) drain_loads();
+  // before exit: the last tile's MMAs and the peer's copy into this CTA have
+  // completed (also when a wait above ran out)
+  if (etid == 0 && it > 0) {
+    volatile int never = 0;
+    mbar_wait(&ctl.accfull, static_cast<uint32_t>(it - 1) & 1u, 1000000000ull, &never);
+    mbar_wait(&ctl.rbar, static_cast<uint32_t>(it - 1) & 1u, 1000000000ull, &never);
+  }
+  if (etid == 0 && it > 0 && lora && ctl.b_dense) {
+    // the last tile's B' rows (issued by this thread whenever a row existed)
+    volatile int never = 0;
+    const int64_t nl = static_cast<int64_t>(pair + (it - 1) * npairs) * tile_rows + keep_lo;
+    if (keep_cols > 0 && nl < N)
+      mbar_wait(&ctl.bbar, static_cast<uint32_t>(it - 1) & 1u, 1000000000ull, &never);
+  }
+  cluster_wait();
+  group_bar(kBarEpi, kDecEpiThreads);
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kDecTmemCols);
   }
 }
 
@@ -714,18 +892,15 @@ cudaError_t launch_decode(const int8_t *Xq, const float *x_scale, const int8_t *
   const int tile_units = static_cast<int>(per < 1 ? 1 : (per > kDecTileUnits ? kDecTileUnits : per));
   const int64_t tiles = (units + tile_units - 1) / tile_units;
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
-  CUtensorMap tm_w, tm_x;
-  memset(&tm_w, 0, sizeof tm_w);
+  CUtensorMap tm_x;
   memset(&tm_x, 0, sizeof tm_x);
-  // K a multiple of 128: one 3D box per operand and stage; otherwise one 2D
-  // box per K block (the last block's tail is filled with zeros)
+  // K a multiple of 128: one 3D Xq box per stage; otherwise one 2D box per K
+  // block (the last block's tail is filled with zeros)
   const int view3d = (K % 128 == 0) ? 1 : 0;
   if (mode != 2) {
-    const bool made =
-        view3d ? (make_tmap_kblocks(&tm_w, Wq, K, N, 8 * tile_units, kDecKbStage) &&
-                  make_tmap_kblocks(&tm_x, Xq, K, M, kDecMaxM, kDecKbStage))
-               : (make_tmap(&tm_w, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, 128, 8 * tile_units) &&
-                  make_tmap(&tm_x, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, 128, kDecMaxM));
+    const bool made = view3d ? make_tmap_kblocks(&tm_x, Xq, K, M, kDecMaxM, kDecKbStage)
+                             : make_tmap(&tm_x, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, 128,
+                                         kDecMaxM);
     if (!made) return cudaErrorInvalidValue;
   }
   cudaLaunchConfig_t cfg = {};
@@ -742,8 +917,8 @@ cudaError_t launch_decode(const int8_t *Xq, const float *x_scale, const int8_t *
   attrs[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = lora ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, decode_gemm_kernel, tm_w, tm_x, view3d, x_scale, w_scale, M, N,
-                            K, mode, B_pack, lora_offset, lora_rank, n_adapters, R, seg_offsets,
+  return cudaLaunchKernelEx(&cfg, decode_gemm_kernel, tm_x, view3d, Wq, x_scale, w_scale, M, N, K,
+                            mode, B_pack, lora_offset, lora_rank, n_adapters, R, seg_offsets,
                             seg_adapter, S, lora ? static_cast<const float *>(part) : nullptr,
                             ksplit, tile_units, static_cast<int>(tiles), out, wait_timeout_ns());
 }

@@ -188,6 +188,25 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint
       : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared through L2 only (no L1
+// allocation); both addresses 16-byte aligned.  The write is a generic-proxy
+// write: a thread that hands the data to the tensor core after observing it
+// through an mbarrier issues fence_proxy_async_shared() first.
+__device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+               : "memory");
+}
+// Arrive once on `bar` when every cp.async this thread issued so far has
+// completed (the arrival is counted in the barrier's expected count).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// Wait until every cp.async this thread issued has completed.
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // 2D tiled bulk-tensor store shared -> global (bulk-group completion).  Parts of
 // the box outside the tensor are not written.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, const void *smem_src, int32_t x,
@@ -342,6 +361,33 @@ __device__ __forceinline__ int2 ld_cluster_i2(uint32_t cluster_addr) {
   asm volatile("ld.shared::cluster.v2.s32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(cluster_addr));
   return v;
 }
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
+// from this CTA's shared memory to shared memory of a CTA of the cluster
+// (`dst_cluster` and `bar_cluster` from mapa); completion counted in bytes on
+// the destination CTA's mbarrier.
+__device__ __forceinline__ void bulk_copy_to_cta(uint32_t dst_cluster, const void *src,
+                                                 uint32_t bytes, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst_cluster),
+      "r"(smem_u32(src)), "r"(bytes), "r"(bar_cluster)
+      : "memory");
+}
+// Prefetch `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *gsrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(gsrc)),
+               "r"(bytes)
+               : "memory");
+}
+// The two halves of a cluster barrier: every thread of the cluster arrives,
+// and waits before its next arrive.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // 4-byte store to shared memory of a CTA of the cluster (address from mapa).
 __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
