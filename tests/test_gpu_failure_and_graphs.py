@@ -39,7 +39,8 @@ def test_wait_on_a_barrier_nothing_sets_times_out():
     assert float((x * 2).sum()) == 8.0  # the context is fine
 
 
-@pytest.mark.parametrize("name", ["parity_ragged", "llama3_8b_oproj_decode_m64_k4096_n4096"])
+@pytest.mark.parametrize("name", ["parity_ragged", "parity_segments",
+                                  "llama3_8b_oproj_decode_m64_k4096_n4096"])
 def test_wait_bound_runs_out_cleanly(name):
     import torch
     import w8a8_smoothquant_int8_b200 as sq

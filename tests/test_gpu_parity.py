@@ -18,7 +18,7 @@ Y_TOL = 1e-2
 DELTA_TOL = 5e-3
 
 SMALL = ["tiny_m16_k256_n256", "parity_ragged", "parity_heavy_f32", "parity_decode",
-         "parity_waves"]
+         "parity_waves", "parity_segments", "parity_segments_large"]
 
 
 def _run(name, **kw):

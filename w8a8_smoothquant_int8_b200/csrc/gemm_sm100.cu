@@ -68,6 +68,12 @@ struct GemmArgs {
   void *out;
   const unsigned long long *lora_mask;  // [ceil(M/16)] 16-column group masks, or null
   int num_mb, num_nb, num_tiles, group_m, num_pairs;
+  // 0: groups of group_m token tiles walk the output-channel tiles; 1: groups
+  // of group_m output-channel tiles walk the token tiles
+  int raster_n;
+  // operand kept in L2 across the walk (loaded with the evict-last policy):
+  // 0 none, 2 Xq
+  int keep;
   uint64_t timeout_ns;
 };
 
@@ -90,15 +96,19 @@ static_assert(sizeof(SharedCtl) <= 1024, "control block fits its 1 KB slot");
 constexpr size_t kSmemBytes = static_cast<size_t>(kStages) * kStageBytes + 1024 + kEpiSmem + 1024;
 
 __device__ __forceinline__ void tile_coords(int tile, const GemmArgs &a, int &mb, int &nb) {
-  // groups of group_m token tiles walk the output-channel tiles together, so
-  // the pairs running at the same time share Xq rows and Wq columns in L2
-  const int per_group = a.group_m * a.num_nb;
+  // groups of group_m tiles of one dimension walk the other dimension
+  // together, so the pairs running at the same time share Xq rows and Wq
+  // columns in L2; the walked operand is the one kept in L2 when it fits
+  const int inner = a.raster_n ? a.num_mb : a.num_nb;
+  const int outer = a.raster_n ? a.num_nb : a.num_mb;
+  const int per_group = a.group_m * inner;
   const int g = tile / per_group;
   const int first = g * a.group_m;
-  const int gm = min(a.num_mb - first, a.group_m);
+  const int gsz = min(outer - first, a.group_m);
   const int local = tile - g * per_group;
-  mb = first + local % gm;
-  nb = local / gm;
+  const int o = first + local % gsz, i = local / gsz;
+  mb = a.raster_n ? i : o;
+  nb = a.raster_n ? o : i;
 }
 
 // The 16-column groups of R that the tile's tokens use: the OR of the words
@@ -258,6 +268,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       const int row_off = static_cast<int>(rank) * kHalf;
+      const uint64_t pol_keep = l2_policy_evict_last();
       bool ok = walk_items(args, pair, nk, [&](int kind, int, int tile, int a, int part, bool,
                                                bool) -> bool {
         if (kind == kNoMain) return true;
@@ -269,7 +280,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t full_pair = map_to_rank(smem_u32(full_local), 0);
         if (rank == 0) mbar_arrive_expect_tx(full_local, 2 * kStageBytes);
         if (kind == kMain) {
-          tma_load_2d_pair(a_dst, &tm_xq, full_pair, a * BK, mb * BM + row_off);
+          if (args.keep == 2)
+            tma_load_2d_pair_hint(a_dst, &tm_xq, full_pair, a * BK, mb * BM + row_off, pol_keep);
+          else
+            tma_load_2d_pair(a_dst, &tm_xq, full_pair, a * BK, mb * BM + row_off);
           tma_load_2d_pair(a_dst + kABytes, &tm_wq, full_pair, a * BK, nb * BN + row_off);
         } else {
           tma_load_2d_pair(a_dst, part ? &tm_tlo : &tm_thi, full_pair, a * kLoraChunk,
@@ -538,6 +552,24 @@ cudaError_t launch_w8a8_gemm(const int8_t *Xq, const int8_t *Wq, const float *x_
   a.num_nb = static_cast<int>((N + BN - 1) / BN);
   a.num_tiles = a.num_mb * a.num_nb;
   a.group_m = 4;
+  // When all of Xq fits half the L2 and Wq does not, groups of
+  // output-channel tiles walk all the token tiles and Xq is loaded with the
+  // evict-last policy: Xq stays, Wq streams through once (measured at
+  // 8192x4096x28672: DRAM reads 1085 -> 361 MB per launch, same time).
+  // Otherwise groups of token tiles walk all output-channel tiles.  (Keeping
+  // Wq the same way at 16384x14336x4096, or walking it in slabs of a
+  // quarter of the L2, did not cut its re-reads and made the kernel slower.)
+  {
+    const double xq_bytes = static_cast<double>(M) * static_cast<double>(K);
+    const double wq_bytes = static_cast<double>(N) * static_cast<double>(K);
+    const double budget = 64.0 * 1024.0 * 1024.0;
+    a.raster_n = 0;
+    a.keep = 0;
+    if (xq_bytes <= budget && wq_bytes > budget) {
+      a.raster_n = 1;
+      a.keep = 2;
+    }
+  }
   a.num_pairs = min(a.num_tiles, sm_count_of_current_device() / 2);
   a.timeout_ns = wait_timeout_ns();
   static std::atomic<int> attr_set[kMaxDevices];

@@ -444,6 +444,25 @@ __device__ __forceinline__ void mma_f16_pair(uint32_t tmem_d, uint64_t adesc, ui
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Same, with an L2 cache-eviction policy for the copied lines (from
+// l2_policy_evict_last).
+__device__ __forceinline__ void tma_load_2d_pair_hint(void *smem_dst, const CUtensorMap *m,
+                                                      uint32_t bar_cluster, int32_t x, int32_t y,
+                                                      uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+// L2 policy: the lines are the last to be evicted (an operand that every
+// tile of a sweep re-reads).
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 // arrive once on `bar` (same shared-memory offset) in every CTA of `cta_mask`
 // when all previously issued MMAs of this thread have completed
 __device__ __forceinline__ void mma_commit_pair(uint64_t *bar, uint16_t cta_mask) {

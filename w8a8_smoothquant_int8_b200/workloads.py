@@ -112,6 +112,16 @@ SPECS = {
     "parity_waves": WorkloadSpec(
         "parity_waves", 2300, 272, 9200, "bf16", "normal", 6, 20.0, 100.0,
         0.5, 256, (8, 16, 64, 32), "random", 9, 0.2),
+    # short segments (a few tokens each: many 16-token groups with three to
+    # five adapters, so the shrink makes several passes over a group), an
+    # adapter of rank 80 (two 64-column blocks), a ragged K tail; the second
+    # is large enough for the shrink's two-group blocks and 65 GEMM row tiles
+    "parity_segments": WorkloadSpec(
+        "parity_segments", 4800, 272, 320, "bf16", "normal", 6, 20.0, 100.0,
+        0.5, 256, (8, 16, 64, 32, 80), "random", 700, 0.2),
+    "parity_segments_large": WorkloadSpec(
+        "parity_segments_large", 16500, 272, 320, "bf16", "normal", 6, 20.0, 100.0,
+        0.5, 256, (8, 16, 64, 32, 80), "random", 2000, 0.2),
 }
 
 # benchmark workloads in the order they are listed with the benchmark
