@@ -111,8 +111,24 @@ def parse():
 KERNEL_TRAFFIC = {
     "llama3_8b_qkv_m2048_k4096_n6144": {
         "file": "gemm_sm100.cu",
-        "source_sha256": "c6429fb71707a01faa20e1b0b08fb3c3b2e7410a0fc50376fb111933d2470d6c",
-        "bytes": 34068992 + 1645824,
+        "source_sha256": "bddc86184aecdea6f0229daa3e334b286019ae9edbacfc434408135e3b1c6db2",
+        "bytes": 34082816 + 1157888,
+    },
+    "llama3_8b_gateup_m8192_k4096_n28672": {
+        "file": "gemm_sm100.cu",
+        "source_sha256": "bddc86184aecdea6f0229daa3e334b286019ae9edbacfc434408135e3b1c6db2",
+        "bytes": 395806464 + 447846656,
+    },
+    "llama3_8b_down_m16384_k14336_n4096": {
+        "file": "gemm_sm100.cu",
+        "source_sha256": "bddc86184aecdea6f0229daa3e334b286019ae9edbacfc434408135e3b1c6db2",
+        "bytes": 1241112320 + 124009984,
+    },
+    # the layer call: decode_shrink_kernel + decode_gemm_kernel
+    "llama3_8b_oproj_decode_m64_k4096_n4096": {
+        "file": "decode.cu",
+        "source_sha256": "ff6e0775024866cfcbd1b67aa126bc8f9bc0e253d4f0c807f69186b214bf0e84",
+        "bytes": 8672512 + 25540096,
     },
 }
 
