@@ -232,11 +232,13 @@ __global__ void __maxnreg__(96) decode_shrink_kernel(
 //     in one round of loads (a load issued while the SM streams waits behind
 //     the copies in flight; for ranks above 64 T is formed after the K loop
 //     where the stages were);
+//   the B' rows of the channels this CTA keeps are bulk-copied into a region
+//     of their own during the K loop when the tokens read most of each row
+//     (else each thread's B' words are copied after it);
 //   then warps 0-1 move D to shared memory, the channels the peer finishes
 //     go to the peer in one bulk copy counted on its mbarrier, and warps 0-7
 //     finish the channels this CTA keeps, one channel per lane and 8 tokens
-//     per warp (their B' words requested before the peer's partials are
-//     awaited): acc = own + peer partial, delta = T B_a^T,
+//     per warp: acc = own + peer partial, delta = T B_a^T,
 //     Y = bf16(acc*xs*ws + delta).
 // Every wait on another thread is bounded; all threads of both CTAs pass the
 // same barriers in the same order, also after a wait that ran out, and no
@@ -246,7 +248,7 @@ __global__ void __maxnreg__(96) decode_shrink_kernel(
 constexpr int kDecTileUnits = 8;                     // 8-channel groups per tile, at most
 constexpr int kDecRowsMax = 8 * kDecTileUnits;       // 64 output channels
 constexpr int kDecKbStage = 2;                       // 128-byte K blocks per stage
-constexpr int kDecStages = 5;
+constexpr int kDecStages = 4;
 constexpr int kDecWBytes = kDecKbStage * kDecRowsMax * 128;  // Wq slabs of a stage (16 KB)
 constexpr int kDecXBytes = kDecKbStage * kDecMaxM * 128;     // Xq slabs of a stage (16 KB)
 constexpr int kDecStageBytes = kDecWBytes + kDecXBytes;
@@ -267,16 +269,16 @@ constexpr uint32_t kDecIdesc = idesc_i8_s32(128, kDecMaxM);
 // full barrier of a stage: one cp.async arrival per loader thread; the Xq
 // box of the stage is counted on a barrier of its own (xfull)
 // after the K loop the ring holds the partials sent to the peer [64][peer
-// channels], this CTA's own partials [64][32], T [64][rank padded to 16]
-// when it has no room of its own, and the epilogue's B' words: either the
-// kept channels' whole B' rows (row stride 2R + 16 bytes, so that lanes on
-// consecutive rows hit distinct banks) or 16 words of 16 bytes per thread,
-// stored [word][thread]
+// channels], this CTA's own partials [64][32] and T [64][rank padded to 16]
+// when it has no room of its own
 constexpr int kDecSendOff = 0, kDecOwnOff = 8192, kDecTOff = 16384;
-constexpr int kDecBOff = kDecTOff + kDecMaxM * kDecMaxRank * 4;
-static_assert(kDecBOff + 16 * kDecEpiThreads * 16 <= kDecRingBytes, "T and B' must fit the ring");
-static_assert(kDecBOff + kDecKeepMax * (2 * SQ_MAX_LORA_COLS + 16) <= kDecRingBytes,
-              "the kept B' rows must fit the ring");
+static_assert(kDecTOff + kDecMaxM * kDecMaxRank * 4 <= kDecRingBytes, "T must fit the ring");
+// the epilogue's B' words have a region of their own: either the kept
+// channels' whole B' rows (copied during the K loop; row stride 2R + 16
+// bytes, so that lanes on consecutive rows hit distinct banks) or 16 words of
+// 16 bytes per thread, stored [word][thread]
+constexpr int kDecBBytes = kDecKeepMax * (2 * SQ_MAX_LORA_COLS + 16);
+static_assert(16 * kDecEpiThreads * 16 <= kDecBBytes, "the per-thread B' words fit the region");
 // the MMA of K block 1 reads 128 rows from its slab: still inside the stage
 static_assert((kDecKbStage - 1) * kDecRowsMax * 128 + 128 * 128 <= kDecStageBytes,
               "the channel rows an MMA reads must stay inside its stage");
@@ -302,7 +304,7 @@ struct DecodeCtl {
 };
 
 constexpr size_t kDecSmemBytes = static_cast<size_t>(kDecRingBytes) + kDecRecvBytes +
-                                 kDecTEarlyBytes + sizeof(DecodeCtl) + 1024;
+                                 kDecTEarlyBytes + kDecBBytes + sizeof(DecodeCtl) + 1024;
 
 // 8 bf16 (one 16-byte word) times 8 fp32 values, added to d in order
 __device__ __forceinline__ float dot8_bf16(const uint4 &w, const float4 &t0, const float4 &t1,
@@ -407,8 +409,9 @@ __global__ void __maxnreg__(96) decode_gemm_kernel(
                                               ~static_cast<uintptr_t>(1023));
   int *recv = reinterpret_cast<int *>(ring + kDecRingBytes);
   float *t_own = reinterpret_cast<float *>(ring + kDecRingBytes + kDecRecvBytes);
-  DecodeCtl &ctl =
-      *reinterpret_cast<DecodeCtl *>(ring + kDecRingBytes + kDecRecvBytes + kDecTEarlyBytes);
+  uint8_t *bst = ring + kDecRingBytes + kDecRecvBytes + kDecTEarlyBytes;  // the B' region
+  DecodeCtl &ctl = *reinterpret_cast<DecodeCtl *>(ring + kDecRingBytes + kDecRecvBytes +
+                                                  kDecTEarlyBytes + kDecBBytes);
   int *sendp = reinterpret_cast<int *>(ring + kDecSendOff);
   int *own = reinterpret_cast<int *>(ring + kDecOwnOff);
   volatile int *abort_flag = &ctl.abort;
@@ -553,14 +556,19 @@ __global__ void __maxnreg__(96) decode_gemm_kernel(
   }
 
   // ------------------------------------------------ MMA, lookup, epilogue
-  // B' rows of a tile's kept channels into L2 ahead of the epilogue, when the
-  // tokens read most of each row
-  auto prefetch_b = [&](int64_t n0) {
+  // the B' rows of a tile's kept channels into their region, while the K
+  // loop runs, when the tokens read most of each row (issued by warp 1,
+  // lane 0; the region is free: the previous tile's epilogue has ended)
+  const uint32_t brow_stride = static_cast<uint32_t>(R * 2 + 16);
+  auto load_b_rows = [&](int64_t n0) {
     const int64_t c0 = n0 + keep_lo;
-    const int64_t rows =
-        max(static_cast<int64_t>(0), min(static_cast<int64_t>(keep_cols), N - c0));
-    if (ctl.b_dense && rows > 0)
-      bulk_prefetch_l2(B_pack + c0 * R, static_cast<uint32_t>(rows * R * 2));
+    const int rows = static_cast<int>(
+        max(static_cast<int64_t>(0), min(static_cast<int64_t>(keep_cols), N - c0)));
+    if (!(lora && ctl.b_dense) || rows <= 0) return;
+    mbar_arrive_expect_tx(&ctl.bbar, static_cast<uint32_t>(rows * R * 2));
+    for (int i = 0; i < rows; ++i)
+      bulk_load(bst + i * brow_stride, B_pack + (c0 + i) * R, static_cast<uint32_t>(R * 2),
+                &ctl.bbar);
   };
   const int etid = threadIdx.x;  // 0..255
   int mq = 0;                    // stages consumed by the MMA thread (all tiles)
@@ -654,7 +662,7 @@ __global__ void __maxnreg__(96) decode_gemm_kernel(
           ctl.rmax = r;
           ctl.b_dense = lora && r > 0 && 2 * 16 * (__popc(used_lo) + __popc(used_hi)) >= R;
           ctl.t_early = ((r + 15) & ~15) <= kDecTEarlyCols;
-          prefetch_b(n0);
+          load_b_rows(n0);
         }
       }
       group_bar(kBarLookup, kDecLookupThreads);
@@ -664,7 +672,7 @@ __global__ void __maxnreg__(96) decode_gemm_kernel(
                           kDecLookupThreads);
       }
     }
-    if (warp == 1 && lane == 0 && it > 0) prefetch_b(n0);
+    if (warp == 1 && lane == 0 && it > 0) load_b_rows(n0);
     group_bar(kBarEpi, kDecEpiThreads);
     const int rmax = ctl.rmax;
     const int tstride = (rmax + 15) & ~15;
@@ -725,18 +733,10 @@ __global__ void __maxnreg__(96) decode_gemm_kernel(
     // the B' words go out before the peer's partials are awaited: whole
     // rows by bulk copies when the tokens read most of them, else each
     // thread's words by cp.async
-    uint8_t *bst = ring + kDecBOff;
     const bool b_rows = lora && ctl.b_dense;
-    const uint32_t brow_stride = static_cast<uint32_t>(R * 2 + 16);
     const int b_nrows =
         static_cast<int>(max(static_cast<int64_t>(0),
                              min(static_cast<int64_t>(keep_cols), N - (n0 + keep_lo))));
-    if (b_rows && etid == 0 && b_nrows > 0) {
-      mbar_arrive_expect_tx(&ctl.bbar, static_cast<uint32_t>(b_nrows * R * 2));
-      for (int i = 0; i < b_nrows; ++i)
-        bulk_load(bst + i * brow_stride, B_pack + (n0 + keep_lo + i) * R,
-                  static_cast<uint32_t>(R * 2), &ctl.bbar);
-    }
     const bool b_staged = lora && !b_rows && rmax <= 16;
     if (live && b_staged) decode_stage_b(bst, etid, brow, 8 * warp, 0, mt, ctl);
     if (!mbar_wait(&ctl.rbar, static_cast<uint32_t>(it) & 1u, timeout_ns, abort_flag)) {
@@ -804,7 +804,7 @@ __global__ void __maxnreg__(96) decode_gemm_kernel(
     mbar_wait(&ctl.accfull, static_cast<uint32_t>(it - 1) & 1u, 1000000000ull, &never);
     mbar_wait(&ctl.rbar, static_cast<uint32_t>(it - 1) & 1u, 1000000000ull, &never);
   }
-  if (etid == 0 && it > 0 && lora && ctl.b_dense) {
+  if (etid == 32 && it > 0 && lora && ctl.b_dense) {
     // the last tile's B' rows (issued by this thread whenever a row existed)
     volatile int never = 0;
     const int64_t nl = static_cast<int64_t>(pair + (it - 1) * npairs) * tile_rows + keep_lo;
