@@ -127,8 +127,8 @@ KERNEL_TRAFFIC = {
     # the layer call: decode_shrink_kernel + decode_gemm_kernel
     "llama3_8b_oproj_decode_m64_k4096_n4096": {
         "file": "decode.cu",
-        "source_sha256": "ff6e0775024866cfcbd1b67aa126bc8f9bc0e253d4f0c807f69186b214bf0e84",
-        "bytes": 8672512 + 25540096,
+        "source_sha256": "303cf96cc6ba475c9509c595f2b8466d4e030b25a52bd6ec6694955e74ca76d7",
+        "bytes": 8672256 + 25544192,
     },
 }
 
