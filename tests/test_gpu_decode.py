@@ -5,8 +5,9 @@ pairs that split K, with the pair's int32 halves added through distributed
 shared memory).  These cases walk its shapes and tables: one token to 64;
 N from one 16-channel group to several tiles per pair; K of one stage, a
 ragged last stage and the shrink's K slices up to their cap; adapters used
-by most tokens (B' staged in shared memory) and by few (B' read from global
-memory); ranks 8 to 256; segments with no adapter, segment tables that are
+by most tokens (whole B' rows copied into shared memory during the K loop)
+and by few (each thread's B' words copied for ranks up to 16, read from
+global memory above); ranks 8 to 256; segments with no adapter, segment tables that are
 not sorted or overlap (the first segment holding a token wins), more
 segments than threads, and more adapters than the staged table holds.
 Bars: int32 accumulators bit-exact, Y within 1e-2 and the delta within 5e-3
@@ -113,7 +114,7 @@ def test_decode_shapes_per_token_adapters(M, N, K):
 
 def test_decode_dense_pack_of_64_adapters():
     # every token its own rank-16 adapter: the B' rows of each CTA's channels
-    # are staged in shared memory
+    # are copied into shared memory during the K loop
     seg, ad = _per_token(64, 64)
     _check(64, 1024, 2048, [16] * 64, seg, ad, pack=([16 * a for a in range(64)], 1024,
                                                      list(range(64))))
@@ -124,6 +125,14 @@ def test_decode_sparse_use_reads_b_from_global():
     seg, ad = [0, 64], [37]
     _check(64, 512, 1024, [16] * 64, seg, ad, pack=([16 * a for a in range(64)], 1024,
                                                     list(range(64))))
+
+
+def test_decode_sparse_use_of_a_wide_adapter_reads_b_from_global():
+    # a 1024-column pack of sixteen rank-64 adapters of which the tokens use
+    # two: too few columns for whole rows, ranks too wide for the copied words
+    seg, ad = [0, 20, 64], [5, 11]
+    _check(64, 400, 1040, [64] * 16, seg, ad, pack=([64 * a for a in range(16)], 1024,
+                                                    list(range(16))))
 
 
 def test_decode_mixed_ranks_and_none():
