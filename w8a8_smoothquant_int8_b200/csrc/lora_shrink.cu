@@ -25,6 +25,8 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "ptx_sm100.cuh"
+#include "tmap.cuh"
 
 namespace sq {
 
@@ -315,6 +317,552 @@ __global__ void __launch_bounds__(kShrinkThreads) lora_shrink_kernel(
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-memory form (large M, quantized input).  The warp-level MMAs above
+// run on the legacy tensor path, which on this GPU sustains only a few
+// hundred multiply-adds per clock per SM: at the largest workloads the form
+// above is bound by it (measured: the same ~1 us per 64-wide K slice per warp
+// whatever the loading scheme).  Here one CTA takes 128 tokens and a range of
+// K in 128-wide slices:
+//  - the lanes of a producer warp load each slice of Xq (int8, 128-byte rows,
+//    128-byte swizzle) and of the A_pack rows of every adapter the 128 tokens
+//    use (two 64-wide halves) into a ring of shared-memory stages with TMA;
+//  - eight converter warps (half a row per thread) turn the int8 slice into
+//    bf16 (exact: |q| <= 128) in the K-major 128-byte-swizzled layout that
+//    tcgen05.mma reads, into one of two slice buffers;
+//  - one thread issues tcgen05.mma kind::f16 (M = 128 tokens, K = 16) with
+//    fp32 accumulators in tensor memory, one 32-column slot per (adapter, 32
+//    columns of it): a single sweep over K serves every adapter of the block
+//    (up to kTSlots slots per sweep), and one MMA of N = 32 x slots covers
+//    all of them (the slots' A_pack rows are contiguous in the stage).  The
+//    eight K steps of a slice accumulate into separate banks (when tensor
+//    memory allows), so that the small MMAs do not wait on one another; the
+//    banks are added when a slot is read back;
+//  - four of the converter warps read the accumulators back (tcgen05.ld);
+//    all of them keep the rows that use each slot's adapter and scale by
+//    x_scale.
+// K is split over the `nsplit` CTAs of a thread-block cluster that share 128
+// tokens: each leaves its fp32 sums in its own shared memory, and each CTA
+// then adds, for its share of the rows, the sums of all CTAs of the cluster
+// in rank order (distributed shared memory), so the result does not depend
+// on timing.  Output as in the form above.
+// ---------------------------------------------------------------------------
+constexpr int kTRows = 128;                     // tokens per CTA (the MMA's M)
+constexpr int kTK = 128;                        // K per stage (one 128-byte Xq row)
+constexpr int kTSlotCols = 32;                  // TMEM columns per slot
+constexpr int kTSlots = 5;                      // slots per sweep over K
+constexpr int kTTmemCols = 256;                 // >= kTSlots * kTSlotCols, a power of 2
+constexpr int kTXBytes = kTRows * kTK;          // int8 slice: 16 KB
+constexpr int kTSlotBytes = kTSlotCols * kTK * 2;  // A_pack slice of one slot: 8 KB (two 64-wide halves)
+constexpr int kTABytes = kTRows * kTK * 2;      // bf16 slice: 32 KB (two 64-wide halves)
+constexpr int kTABufs = 2;
+constexpr int kTMaxStages = 8;
+constexpr int kTSmem = 216 * 1024;              // dynamic shared memory (one CTA per SM)
+constexpr int kTConvWarps = 8;                  // two per row quarter of the slice
+constexpr int kTThreads = (2 + kTConvWarps) * 32;  // producer, MMA, converter/epilogue warps
+constexpr int kTMaxPasses = kTRows * (SQ_MAX_LORA_RANK / kTSlotCols);
+constexpr int kTTargetCtas = 148;               // split K until about this many CTAs
+constexpr int kTMaxSplit = 8;                   // CTAs of a cluster (portable size)
+constexpr int kTMinSlicesPerSplit = 8;
+constexpr int kTTab = 1024;                     // segment / adapter tables staged in smem
+
+// K splits for M tokens: about kTTargetCtas CTAs in all, at most a portable
+// cluster, and at least kTMinSlicesPerSplit K slices per split.
+static inline int tc_shrink_splits(int64_t M) {
+  const int64_t nrb = (M + kTRows - 1) / kTRows;
+  int64_t n = kTTargetCtas / (nrb > 0 ? nrb : 1);
+  return static_cast<int>(n < 1 ? 1 : (n > kTMaxSplit ? kTMaxSplit : n));
+}
+
+struct ShrinkPass {
+  int16_t row;  // first row of the block with the pass's adapter
+  int16_t cb;   // first adapter column of the pass
+};
+
+struct ShrinkCtl {
+  uint64_t full[kTMaxStages], empty[kTMaxStages];  // ring: TMA -> (converters, MMA)
+  uint64_t afull[kTABufs], aempty[kTABufs];        // bf16 slices: converters <-> MMA
+  uint64_t done, tfree, drain;                     // accumulators ready / read / MMAs retired
+  uint32_t tmem_base;
+  int abort, npass;
+  int ad[kTRows], off[kTRows], rank[kTRows], groups[kTRows];
+  ShrinkPass pass[kTMaxPasses];
+};
+
+// 8 consecutive T values of a row -> the 16-byte words of both planes.
+__device__ __forceinline__ void store_t8(uint16_t *T_hi, uint16_t *T_lo, int64_t idx,
+                                         const float (&v)[8]) {
+  uint32_t hi[4], lo[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * j]), h1 = __float2bfloat16_rn(v[2 * j + 1]);
+    const __nv_bfloat16 l0 = __float2bfloat16_rn(v[2 * j] - __bfloat162float(h0));
+    const __nv_bfloat16 l1 = __float2bfloat16_rn(v[2 * j + 1] - __bfloat162float(h1));
+    hi[j] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+            (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+    lo[j] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
+            (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+  }
+  *reinterpret_cast<uint4 *>(T_hi + idx) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  *reinterpret_cast<uint4 *>(T_lo + idx) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+}
+
+
+// Rows of the 128-token block handled by cluster rank q in the reduction.
+__device__ __forceinline__ void share_rows(int q, int ns, int &lo, int &hi) {
+  lo = q * kTRows / ns;
+  hi = (q + 1) * kTRows / ns;
+}
+
+__global__ void __launch_bounds__(kTThreads, 1) lora_shrink_tc_kernel(
+    const __grid_constant__ CUtensorMap tm_xq, const __grid_constant__ CUtensorMap tm_a,
+    const float *__restrict__ x_scale, int64_t M, int64_t K,
+    const int32_t *__restrict__ lora_offset, const int32_t *__restrict__ lora_rank,
+    int n_adapters, int64_t R, const int32_t *__restrict__ seg_offsets,
+    const int32_t *__restrict__ seg_adapter, int64_t S, int nsplit, uint16_t *__restrict__ T_hi,
+    uint16_t *__restrict__ T_lo, unsigned long long *__restrict__ mask, uint64_t timeout_ns) {
+  extern __shared__ uint8_t sh_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sh_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  __shared__ ShrinkCtl ctl;
+  volatile int *abort_flag = &ctl.abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rb = blockIdx.x / nsplit, sp = blockIdx.x - rb * nsplit;  // sp: rank in the cluster
+  const int64_t row0 = static_cast<int64_t>(rb) * kTRows;
+  const int nslices = static_cast<int>((K + kTK - 1) / kTK);
+  const int c0 = static_cast<int>(static_cast<int64_t>(sp) * nslices / nsplit);
+  const int c1 = static_cast<int>(static_cast<int64_t>(sp + 1) * nslices / nsplit);
+
+  // ---- segment and adapter tables into shared memory (the stage area is
+  //      not in use yet), then each row's adapter, column offset and rank
+  int32_t *t_seg = reinterpret_cast<int32_t *>(base);  // S + 1 offsets
+  int32_t *t_sad = t_seg + kTTab + 1;                  // S adapters
+  int32_t *t_off = t_sad + kTTab;                      // lora_offset
+  int32_t *t_rnk = t_off + kTTab;                      // lora_rank
+  const bool seg_tab = S <= kTTab, ad_tab = n_adapters <= kTTab;
+  if (seg_tab)
+    for (int i = threadIdx.x; i <= static_cast<int>(S); i += kTThreads) {
+      t_seg[i] = seg_offsets[i];
+      if (i < S) t_sad[i] = seg_adapter[i];
+    }
+  if (ad_tab)
+    for (int i = threadIdx.x; i < n_adapters; i += kTThreads) {
+      t_off[i] = lora_offset[i];
+      t_rnk[i] = lora_rank[i];
+    }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kTMaxStages; ++i) {
+      mbar_init(&ctl.full[i], 1);
+      mbar_init(&ctl.empty[i], kTConvWarps + 1);  // the converter warps and the MMA commit
+    }
+    for (int i = 0; i < kTABufs; ++i) {
+      mbar_init(&ctl.afull[i], kTConvWarps);
+      mbar_init(&ctl.aempty[i], 1);
+    }
+    mbar_init(&ctl.done, 1);
+    mbar_init(&ctl.tfree, 4);
+    mbar_init(&ctl.drain, 1);
+    ctl.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctl.tmem_base, kTTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x < kTRows) {
+    const int64_t i = row0 + threadIdx.x;
+    int a = (i < M) ? token_adapter(seg_tab ? t_seg : seg_offsets, seg_tab ? t_sad : seg_adapter,
+                                    S, n_adapters, i)
+                    : -1;
+    int off = 0, r = 0;
+    if (a >= 0) {
+      off = ad_tab ? t_off[a] : lora_offset[a];
+      r = ad_tab ? t_rnk[a] : lora_rank[a];
+      if (off < 0 || (off & 15) || r <= 0 || r > SQ_MAX_LORA_RANK || off + ((r + 15) & ~15) > R) {
+        record_device_error(SQ_ERR_BAD_SEGMENTS);
+        a = -1;
+        off = 0;
+        r = 0;
+      }
+    }
+    ctl.ad[threadIdx.x] = a;
+    ctl.off[threadIdx.x] = off;
+    ctl.rank[threadIdx.x] = r;
+  }
+  __syncthreads();
+  // passes: one per (adapter, 32 columns of it), adapters in order of first
+  // appearance among the rows (the same in every CTA of the cluster)
+  if (threadIdx.x < kTRows) {
+    const int a = ctl.ad[threadIdx.x];
+    bool first = a >= 0;
+    for (int j = 0; j < static_cast<int>(threadIdx.x) && first; ++j) first = ctl.ad[j] != a;
+    const int rpad = (ctl.rank[threadIdx.x] + 15) & ~15;
+    ctl.groups[threadIdx.x] = first ? (rpad + kTSlotCols - 1) / kTSlotCols : 0;
+  }
+  __syncthreads();
+  {
+    // pass indices: an exclusive prefix sum of the groups over the rows
+    __shared__ int wsum[kTRows / 32];
+    const int g = (threadIdx.x < kTRows) ? ctl.groups[threadIdx.x] : 0;
+    int incl = g;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (threadIdx.x < kTRows && lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (threadIdx.x < kTRows) {
+      int excl = incl - g;
+      for (int w = 0; w < warp; ++w) excl += wsum[w];
+      for (int gi = 0; gi < g; ++gi)
+        ctl.pass[excl + gi] = ShrinkPass{static_cast<int16_t>(threadIdx.x),
+                                         static_cast<int16_t>(gi * kTSlotCols)};
+      if (threadIdx.x == kTRows - 1) ctl.npass = excl + g;
+    }
+  }
+  __syncthreads();
+  // the tokens' codes and scales come from the preceding kernel (programmatic
+  // dependent launch: everything above overlapped its tail)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int npass = ctl.npass;
+  const int nsweep = (npass + kTSlots - 1) / kTSlots;
+  const int slots_max = npass < kTSlots ? npass : kTSlots;
+  const int stage_bytes = kTXBytes + slots_max * kTSlotBytes;
+  // bf16 slices in flight between the converters and the MMAs, then the ring
+  const int nab = kTABufs;
+  int stages = (kTSmem - 1024 - nab * kTABytes) / stage_bytes;
+  stages = stages > kTMaxStages ? kTMaxStages : stages;
+  uint8_t *abuf = base;                   // nab bf16 slices
+  uint8_t *ring = base + nab * kTABytes;  // stages: int8 slice + A_pack slots
+  // independent accumulator banks: the K steps of a slice go to different
+  // banks, so consecutive MMAs do not wait on each other; summed at the end
+  const int nbank = (slots_max <= 2) ? 4 : ((slots_max <= 4) ? 2 : 1);
+  const uint32_t tmem = ctl.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int st = 0;
+    uint32_t ph = 0;
+    int64_t issued = 0;
+    for (int sw = 0; sw < nsweep; ++sw) {
+      const int p0 = sw * kTSlots, np = min(kTSlots, npass - p0);
+      if (sw == 0 && lane == 0) {
+        prefetch_tmap(&tm_xq);
+        prefetch_tmap(&tm_a);
+      }
+      // copies of a stage: lane 0 the Xq box, lanes 1.. the A_pack boxes
+      // (slot q, half h, 16-row group g16); several lanes issue together
+      int ncopy = 1;
+      uint32_t bytes = kTXBytes;
+      for (int q = 0; q < np; ++q) {
+        const int i = ctl.pass[p0 + q].row, cb = ctl.pass[p0 + q].cb;
+        const int w = min(kTSlotCols, ((ctl.rank[i] + 15) & ~15) - cb);
+        ncopy += 2 * (w / 16);
+        bytes += static_cast<uint32_t>(w) * kTK * 2;
+      }
+      int my_q = -1, my_h = 0, my_g = 0;
+      if (lane >= 1 && lane < ncopy) {
+        int k = lane - 1;
+        for (int q = 0; q < np && my_q < 0; ++q) {
+          const int i = ctl.pass[p0 + q].row, cb = ctl.pass[p0 + q].cb;
+          const int n2 = 2 * (min(kTSlotCols, ((ctl.rank[i] + 15) & ~15) - cb) / 16);
+          if (k < n2) {
+            my_q = q;
+            my_h = k / (n2 / 2);
+            my_g = k % (n2 / 2);
+          } else {
+            k -= n2;
+          }
+        }
+      }
+      for (int c = c0; c < c1; ++c) {
+        bool go = false;
+        if (lane == 0) {
+          go = !*abort_flag && mbar_wait(&ctl.empty[st], ph ^ 1u, timeout_ns, abort_flag);
+          if (!go) {
+            *abort_flag = 1;
+            record_device_error(SQ_ERR_DEVICE_TIMEOUT);
+          } else {
+            mbar_arrive_expect_tx(&ctl.full[st], bytes);
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, go, 0)) break;
+        uint8_t *dst = ring + st * stage_bytes;
+        if (lane == 0) tma_load_2d(dst, &tm_xq, &ctl.full[st], c * kTK, static_cast<int32_t>(row0));
+        if (my_q >= 0) {
+          const int i = ctl.pass[p0 + my_q].row, cb = ctl.pass[p0 + my_q].cb;
+          tma_load_2d(dst + kTXBytes + my_h * (slots_max * kTSlotCols * 128) +
+                          my_q * (kTSlotCols * 128) + my_g * 2048,
+                      &tm_a, &ctl.full[st], c * kTK + 64 * my_h, ctl.off[i] + cb + 16 * my_g);
+        }
+        ++issued;
+        if (++st == stages) { st = 0; ph ^= 1u; }
+      }
+      __syncwarp();
+      // the sweep's sums are exchanged through the stage area, which is
+      // refilled only after both cluster barriers
+      cluster_sync();
+      cluster_sync();
+    }
+    if (lane == 0) {
+      // every copy issued must land before the block exits
+      volatile int never = 0;
+      for (int s2 = 0; s2 < stages && s2 < issued; ++s2) {
+        const int64_t last = issued - 1 - ((issued - 1 - s2) % stages);
+        mbar_wait(&ctl.full[s2], static_cast<uint32_t>((last / stages) & 1), 1000000000ull, &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    int st = 0, b = 0;
+    uint32_t ph = 0, bph = 0;
+    for (int sw = 0; sw < nsweep; ++sw) {
+      const int p0 = sw * kTSlots, np = min(kTSlots, npass - p0);
+      if (lane == 0) {
+        tc_fence_after();  // the previous sweep's accumulators have been read
+        bool ok = !*abort_flag;
+        for (int c = c0; c < c1 && ok; ++c) {
+          if (!mbar_wait(&ctl.afull[b], bph, timeout_ns, abort_flag) ||
+              !mbar_wait(&ctl.full[st], ph, timeout_ns, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(abuf + b * kTABytes);
+          const uint32_t s_addr = smem_u32(ring + st * stage_bytes + kTXBytes);
+          // one MMA per K step for all slots of the sweep: their A_pack rows
+          // are contiguous within each 64-wide half (a slot narrower than 32
+          // columns leaves rows that only its own unused columns read)
+          const uint32_t idesc = idesc_bf16_f32(kTRows, static_cast<uint32_t>(np * kTSlotCols));
+#pragma unroll
+          for (int kk = 0; kk < kTK / 16; ++kk) {
+            const int h = kk >> 2, k16 = kk & 3;  // 64-wide half, K step inside it
+            const int bank = kk % nbank;
+            mma_f16(tmem + static_cast<uint32_t>(bank * slots_max * kTSlotCols),
+                    sdesc_kmajor_sw128(a_addr + h * (kTRows * 128) + 32 * k16),
+                    sdesc_kmajor_sw128(s_addr + h * (slots_max * kTSlotCols * 128) + 32 * k16),
+                    idesc, (c > c0 || kk >= nbank) ? 1u : 0u);
+          }
+          mma_commit(&ctl.aempty[b]);
+          mma_commit(&ctl.empty[st]);
+          if (++st == stages) { st = 0; ph ^= 1u; }
+          if (++b == nab) { b = 0; bph ^= 1u; }
+        }
+        if (ok) {
+          mma_commit(&ctl.done);
+        } else if (!*abort_flag) {
+          *abort_flag = 1;
+          record_device_error(SQ_ERR_DEVICE_TIMEOUT);
+        }
+      }
+      __syncwarp();
+      cluster_sync();
+      cluster_sync();
+    }
+    if (lane == 0 && nsweep > 0) {
+      // every MMA issued must retire before TMEM is freed
+      mma_commit(&ctl.drain);
+      volatile int never = 0;
+      mbar_wait(&ctl.drain, 0, 1000000000ull, &never);
+    }
+  } else {
+    // ------------------------------------------- converters, then epilogue
+    const int ctid = threadIdx.x - 64;     // 0..255 among the converter threads
+    const int r = ctid & (kTRows - 1);     // row converted by this thread
+    const int hq = ctid >> 7;              // its half of the row: int8 chunks 4hq .. 4hq+3
+    const int quarter = warp & 3;          // TMEM lanes of this warp
+    const int re = quarter * 32 + lane;    // row read back by this thread
+    int st = 0, b = 0;
+    uint32_t ph = 0, bph = 0;
+    int lo_row, hi_row;
+    share_rows(sp, nsplit, lo_row, hi_row);
+    for (int sw = 0; sw < nsweep; ++sw) {
+      const int p0 = sw * kTSlots, np = min(kTSlots, npass - p0);
+      bool ok = !*abort_flag;
+      for (int c = c0; c < c1 && ok; ++c) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&ctl.full[st], ph, timeout_ns, abort_flag)) &&
+             __all_sync(0xffffffffu, mbar_wait(&ctl.aempty[b], bph ^ 1u, timeout_ns, abort_flag));
+        if (!ok) break;
+        // row r: 128 int8 codes (128-byte swizzle: chunk q at q ^ (r & 7));
+        // this thread's chunks 4hq .. 4hq+3 are the codes of the slice's
+        // 64-wide half hq, written as that half's bf16 row
+        const uint8_t *src = ring + st * stage_bytes + r * 128;
+        uint8_t *dst = abuf + b * kTABytes + hq * (kTRows * 128) + r * 128;
+        uint4 v[4];
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq)
+          v[qq] = *reinterpret_cast<const uint4 *>(src + (((4 * hq + qq) ^ (r & 7)) * 16));
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const uint32_t w4[4] = {v[qq].x, v[qq].y, v[qq].z, v[qq].w};
+          // bf16 chunks 2qq (codes 16qq..16qq+7 of the half) and 2qq+1
+          const uint4 c_lo = make_uint4(bf16x2_of_s8(w4[0], 0), bf16x2_of_s8(w4[0], 2),
+                                        bf16x2_of_s8(w4[1], 0), bf16x2_of_s8(w4[1], 2));
+          const uint4 c_hi = make_uint4(bf16x2_of_s8(w4[2], 0), bf16x2_of_s8(w4[2], 2),
+                                        bf16x2_of_s8(w4[3], 0), bf16x2_of_s8(w4[3], 2));
+          *reinterpret_cast<uint4 *>(dst + (((2 * qq) ^ (r & 7)) * 16)) = c_lo;
+          *reinterpret_cast<uint4 *>(dst + (((2 * qq + 1) ^ (r & 7)) * 16)) = c_hi;
+        }
+        fence_proxy_async_shared();  // the tensor core reads the slice
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&ctl.afull[b]);
+          mbar_arrive(&ctl.empty[st]);
+        }
+        if (++st == stages) { st = 0; ph ^= 1u; }
+        if (++b == nab) { b = 0; bph ^= 1u; }
+      }
+      // this CTA's sums -> its shared memory, slot q at base + q * 16 KB,
+      // row-major 128-byte rows (16-byte chunk c of row x at c ^ (x & 7))
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&ctl.done, static_cast<uint32_t>(sw & 1),
+                                                     timeout_ns, abort_flag));
+      if (!ok) {
+        if (!*abort_flag) {
+          *abort_flag = 1;
+          record_device_error(SQ_ERR_DEVICE_TIMEOUT);
+        }
+      } else if (ctid < kTRows) {  // warps 2-5 cover the four lane quarters
+        tc_fence_after();
+        for (int q = 0; q < np; ++q) {
+          uint8_t *prow = base + q * (kTRows * 128) + re * 128;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float acc16[16];
+            for (int bank = 0; bank < nbank; ++bank) {
+              uint32_t v[16];
+              tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                     static_cast<uint32_t>((bank * slots_max + q) * kTSlotCols + 16 * h),
+                                 v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                acc16[j] = (bank == 0) ? __uint_as_float(v[j]) : acc16[j] + __uint_as_float(v[j]);
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              *reinterpret_cast<uint4 *>(prow + (((4 * h + c) ^ (re & 7)) * 16)) =
+                  make_uint4(__float_as_uint(acc16[4 * c]), __float_as_uint(acc16[4 * c + 1]),
+                             __float_as_uint(acc16[4 * c + 2]), __float_as_uint(acc16[4 * c + 3]));
+          }
+        }
+        tc_fence_before();
+      }
+      __syncwarp();
+      cluster_sync();  // every CTA's sums are in place
+      // rows [lo_row, hi_row): sum over the cluster's CTAs in rank order
+      const int nrow = hi_row - lo_row;
+      for (int e = ctid; e < nrow * np * 4; e += 32 * kTConvWarps) {
+        const int q = e / (nrow * 4), rem = e - q * nrow * 4;
+        const int x = lo_row + rem / 4, c8 = rem % 4;  // row, 8-column group of the slot
+        const int i = ctl.pass[p0 + q].row, cb = ctl.pass[p0 + q].cb;
+        const int a = ctl.ad[i], off = ctl.off[i], rank = ctl.rank[i];
+        const int w = min(kTSlotCols, ((rank + 15) & ~15) - cb);
+        const int64_t row = row0 + x;
+        if (8 * c8 >= w || row >= M || ctl.ad[x] != a || *abort_flag) continue;
+        const uint32_t local = smem_u32(base + q * (kTRows * 128) + x * 128);
+        float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int p0 = 0; p0 < nsplit; p0 += 4) {  // rank order, four loads pairs in flight
+          float4 pv[4][2];
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (p0 + u < nsplit) {
+              const uint32_t ra = map_to_rank(local, static_cast<uint32_t>(p0 + u));
+              pv[u][0] = ld_cluster_f4(ra + (((2 * c8) ^ (x & 7)) * 16));
+              pv[u][1] = ld_cluster_f4(ra + (((2 * c8 + 1) ^ (x & 7)) * 16));
+            }
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (p0 + u < nsplit) {
+              s8[0] += pv[u][0].x; s8[1] += pv[u][0].y; s8[2] += pv[u][0].z; s8[3] += pv[u][0].w;
+              s8[4] += pv[u][1].x; s8[5] += pv[u][1].y; s8[6] += pv[u][1].z; s8[7] += pv[u][1].w;
+            }
+        }
+        const float xs = x_scale[row];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s8[j] = (cb + 8 * c8 + j < rank) ? xs * s8[j] : 0.f;
+        store_t8(T_hi, T_lo, row * R + off + cb + 8 * c8, s8);
+      }
+      __syncwarp();
+      cluster_sync();  // the peers are done reading this CTA's sums
+    }
+    // zeros outside each row's adapter columns, for this CTA's share of rows
+    const int words = static_cast<int>(R / 8);  // 8 columns: 16 bytes of a plane
+    for (int e = ctid; e < (hi_row - lo_row) * words; e += 32 * kTConvWarps) {
+      const int x = lo_row + e / words, wcol = (e % words) * 8;
+      const int64_t row = row0 + x;
+      if (row >= M) continue;
+      const int a = ctl.ad[x], off = ctl.off[x], rpad = (ctl.rank[x] + 15) & ~15;
+      if (a >= 0 && wcol >= off && wcol < off + rpad) continue;
+      *reinterpret_cast<uint4 *>(T_hi + row * R + wcol) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4 *>(T_lo + row * R + wcol) = make_uint4(0, 0, 0, 0);
+    }
+    if (sp == 0 && ctid < kTRows / 16 && row0 + 16 * ctid < M) {
+      // the 16-column groups that each group of 16 tokens uses (one word each)
+      unsigned long long bits = 0;
+      for (int x = 16 * ctid; x < 16 * ctid + 16; ++x) {
+        if (ctl.ad[x] < 0) continue;
+        const int off = ctl.off[x], rpad = (ctl.rank[x] + 15) & ~15;
+        for (int gi = off / 16; gi < (off + rpad) / 16; ++gi) bits |= 1ull << gi;
+      }
+      mask[(row0 >> 4) + ctid] = bits;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTTmemCols);
+  }
+}
+
+
+// Launch of the tensor-memory form: 128-token blocks, K split over a cluster
+// of up to eight CTAs so that about one CTA per SM runs.
+static cudaError_t launch_lora_shrink_tc(const int8_t *Xq, const float *x_scale, int64_t M,
+                                         int64_t K, const uint16_t *A_pack,
+                                         const int32_t *lora_offset, const int32_t *lora_rank,
+                                         int n_adapters, int64_t R, const int32_t *seg_offsets,
+                                         const int32_t *seg_adapter, int64_t S, uint16_t *T_hi,
+                                         uint16_t *T_lo, unsigned long long *mask,
+                                         cudaStream_t st) {
+  const int64_t nrb = (M + kTRows - 1) / kTRows;
+  const int nslices = static_cast<int>((K + kTK - 1) / kTK);
+  int nsplit = tc_shrink_splits(M);
+  const int most = nslices / kTMinSlicesPerSplit;  // keep at least a few slices per split
+  if (nsplit > most) nsplit = most > 1 ? most : 1;
+  CUtensorMap tm_xq, tm_a;
+  memset(&tm_xq, 0, sizeof tm_xq);
+  memset(&tm_a, 0, sizeof tm_a);
+  if (!make_tmap(&tm_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, kTK, kTRows,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap(&tm_a, A_pack, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, R, 64, 16))
+    return cudaErrorInvalidValue;
+  static std::atomic<int> attr_set[kMaxDevices];
+  cudaError_t e = ensure_smem_optin(lora_shrink_tc_kernel, kTSmem, attr_set);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(nrb * nsplit), 1, 1);
+  cfg.blockDim = dim3(kTThreads, 1, 1);
+  cfg.dynamicSmemBytes = kTSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(nsplit);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, lora_shrink_tc_kernel, tm_xq, tm_a, x_scale, M, K, lora_offset,
+                            lora_rank, n_adapters, R, seg_offsets, seg_adapter, S, nsplit, T_hi,
+                            T_lo, mask, wait_timeout_ns());
+}
+
 template <bool kRaw>
 static cudaError_t launch_lora_shrink_t(const void *X, const float *x_scale, int64_t M, int64_t K,
                                         const uint16_t *A_pack, const int32_t *lora_offset,
@@ -375,6 +923,11 @@ cudaError_t launch_lora_shrink(const int8_t *Xq, const float *x_scale, int64_t M
                                uint16_t *T_hi, uint16_t *T_lo, unsigned long long *mask,
                                cudaStream_t st) {
   if (M == 0) return cudaSuccess;
+  // the tensor-memory form once 128-token blocks fill at least half the SMs
+  const int nsm = sm_count_of_current_device();
+  if (nsm > 0 && M >= static_cast<int64_t>(kTRows) * (nsm / 2))
+    return launch_lora_shrink_tc(Xq, x_scale, M, K, A_pack, lora_offset, lora_rank, n_adapters,
+                                 R, seg_offsets, seg_adapter, S, T_hi, T_lo, mask, st);
   return launch_lora_shrink_t<false>(Xq, x_scale, M, K, A_pack, lora_offset, lora_rank,
                                      n_adapters, R, seg_offsets, seg_adapter, S, T_hi, T_lo, mask,
                                      st);
