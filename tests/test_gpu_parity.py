@@ -136,3 +136,20 @@ def test_full_size_sampled(name):
     g.linear()
     assert rel_err(g.Y_f32()[rows], out["Y"]) <= Y_TOL
     assert rel_err(g.delta()[rows], out["delta"]) <= DELTA_TOL
+
+
+# The tensor-memory form of the shrink splits K over a cluster of CTAs when
+# there are few 128-token blocks, as wide as all clusters stay resident at
+# once: 4096 tokens at K=4096 (clusters of four), 6144 tokens (clusters of
+# three would not all be resident: two) and 4096 tokens at K=14336.
+@pytest.mark.parametrize("name,M", [("llama3_8b_gateup_m8192_k4096_n28672", 4096),
+                                    ("llama3_8b_gateup_m8192_k4096_n28672", 6144),
+                                    ("llama3_8b_down_m16384_k14336_n4096", 4096)])
+def test_shrink_cluster_splits_sampled(name, M):
+    from tests.gpu_pipeline import rel_err
+    wl, P, g = _run(name, M=M)
+    rows = _sample_rows(wl.M, np.random.default_rng(11))
+    out = P.rows(rows, want=("Y", "delta"))
+    g.linear()
+    assert rel_err(g.Y_f32()[rows], out["Y"]) <= Y_TOL
+    assert rel_err(g.delta()[rows], out["delta"]) <= DELTA_TOL

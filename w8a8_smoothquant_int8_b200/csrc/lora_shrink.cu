@@ -820,8 +820,36 @@ __global__ void __launch_bounds__(kTThreads, 1) lora_shrink_tc_kernel(
 }
 
 
+// Clusters of `size` CTAs of the tensor-memory form that are resident at
+// once on the current device (asked of the runtime once per device and size).
+static cudaError_t tc_clusters_resident(int size, int *out) {
+  static std::atomic<int> cache[kMaxDevices][kTMaxSplit + 1];
+  const int dev = current_device_index();
+  if (dev < 0 || size < 1 || size > kTMaxSplit) return cudaErrorInvalidValue;
+  int n = cache[dev][size].load(std::memory_order_relaxed);
+  if (n == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(size), 1, 1);
+    cfg.blockDim = dim3(kTThreads, 1, 1);
+    cfg.dynamicSmemBytes = kTSmem;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = static_cast<unsigned>(size);
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, lora_shrink_tc_kernel, &cfg);
+    if (e != cudaSuccess) return e;
+    n = n > 0 ? n + 1 : 1;  // stored plus one: 0 means not asked yet
+    cache[dev][size].store(n, std::memory_order_relaxed);
+  }
+  *out = n - 1;
+  return cudaSuccess;
+}
+
 // Launch of the tensor-memory form: 128-token blocks, K split over a cluster
-// of up to eight CTAs so that about one CTA per SM runs.
+// of up to eight CTAs so that about one CTA per SM runs, all clusters at once.
 static cudaError_t launch_lora_shrink_tc(const int8_t *Xq, const float *x_scale, int64_t M,
                                          int64_t K, const uint16_t *A_pack,
                                          const int32_t *lora_offset, const int32_t *lora_rank,
@@ -834,6 +862,19 @@ static cudaError_t launch_lora_shrink_tc(const int8_t *Xq, const float *x_scale,
   int nsplit = tc_shrink_splits(M);
   const int most = nslices / kTMinSlicesPerSplit;  // keep at least a few slices per split
   if (nsplit > most) nsplit = most > 1 ? most : 1;
+  static std::atomic<int> attr_set[kMaxDevices];
+  cudaError_t e = ensure_smem_optin(lora_shrink_tc_kernel, kTSmem, attr_set);
+  if (e != cudaSuccess) return e;
+  // the widest split whose clusters are all resident at once (one CTA per
+  // SM: clusters of 3 or more CTAs leave SMs of a GPC unused, so fewer of
+  // them fit than SMs / size)
+  while (nsplit > 1) {
+    int fit = 0;
+    e = tc_clusters_resident(nsplit, &fit);
+    if (e != cudaSuccess) return e;
+    if (fit >= nrb) break;
+    --nsplit;
+  }
   CUtensorMap tm_xq, tm_a;
   memset(&tm_xq, 0, sizeof tm_xq);
   memset(&tm_a, 0, sizeof tm_a);
@@ -841,9 +882,6 @@ static cudaError_t launch_lora_shrink_tc(const int8_t *Xq, const float *x_scale,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap(&tm_a, A_pack, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, R, 64, 16))
     return cudaErrorInvalidValue;
-  static std::atomic<int> attr_set[kMaxDevices];
-  cudaError_t e = ensure_smem_optin(lora_shrink_tc_kernel, kTSmem, attr_set);
-  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(nrb * nsplit), 1, 1);
   cfg.blockDim = dim3(kTThreads, 1, 1);
@@ -923,9 +961,11 @@ cudaError_t launch_lora_shrink(const int8_t *Xq, const float *x_scale, int64_t M
                                uint16_t *T_hi, uint16_t *T_lo, unsigned long long *mask,
                                cudaStream_t st) {
   if (M == 0) return cudaSuccess;
-  // the tensor-memory form once 128-token blocks fill at least half the SMs
+  // the tensor-memory form once there are 128-token blocks for a fifth of the
+  // SMs (measured: at 2048 tokens the form above is faster, from 4096 on
+  // this one; K split over clusters fills the remaining SMs)
   const int nsm = sm_count_of_current_device();
-  if (nsm > 0 && M >= static_cast<int64_t>(kTRows) * (nsm / 2))
+  if (nsm > 0 && M >= static_cast<int64_t>(kTRows) * (nsm / 5))
     return launch_lora_shrink_tc(Xq, x_scale, M, K, A_pack, lora_offset, lora_rank, n_adapters,
                                  R, seg_offsets, seg_adapter, S, T_hi, T_lo, mask, st);
   return launch_lora_shrink_t<false>(Xq, x_scale, M, K, A_pack, lora_offset, lora_rank,
