@@ -39,7 +39,7 @@ def test_wait_on_a_barrier_nothing_sets_times_out():
     assert float((x * 2).sum()) == 8.0  # the context is fine
 
 
-@pytest.mark.parametrize("name", ["parity_ragged", "parity_segments",
+@pytest.mark.parametrize("name", ["parity_ragged", "parity_segments", "parity_segments_large",
                                   "llama3_8b_oproj_decode_m64_k4096_n4096"])
 def test_wait_bound_runs_out_cleanly(name):
     import torch

@@ -58,7 +58,7 @@ class RawRun:
                                            wl.seg_offsets, sa, rows, want)
 
 
-SMALL = ["parity_ragged", "parity_decode"]
+SMALL = ["parity_ragged", "parity_decode", "parity_segments_large"]
 
 
 @pytest.fixture(scope="module", params=SMALL)

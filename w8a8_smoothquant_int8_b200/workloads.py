@@ -114,10 +114,13 @@ SPECS = {
         0.5, 256, (8, 16, 64, 32), "random", 9, 0.2),
     # short segments (a few tokens each: many 16-token groups with three to
     # five adapters, so the shrink makes several passes over a group), an
-    # adapter of rank 80 (two 64-column blocks), a ragged K tail; the second
-    # is large enough for the shrink's two-group blocks and 65 GEMM row tiles
+    # adapter of rank 80 (two 64-column blocks), a ragged K tail.  The first
+    # is small enough for the warp-MMA form of the shrink; the second runs
+    # its tensor-memory form (several sweeps over K where a 128-token block
+    # uses more than five 32-column slots), the raw-input form's two-group
+    # blocks, and 65 GEMM row tiles
     "parity_segments": WorkloadSpec(
-        "parity_segments", 4800, 272, 320, "bf16", "normal", 6, 20.0, 100.0,
+        "parity_segments", 3300, 272, 320, "bf16", "normal", 6, 20.0, 100.0,
         0.5, 256, (8, 16, 64, 32, 80), "random", 700, 0.2),
     "parity_segments_large": WorkloadSpec(
         "parity_segments_large", 16500, 272, 320, "bf16", "normal", 6, 20.0, 100.0,
