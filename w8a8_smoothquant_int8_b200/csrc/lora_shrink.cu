@@ -374,6 +374,24 @@ constexpr int kTMaxSplit = 8;                   // CTAs of a cluster (portable s
 constexpr int kTMinSlicesPerSplit = 8;
 constexpr int kTTab = 1024;                     // segment / adapter tables staged in smem
 
+// two converter threads per token row, and the four epilogue warps cover the
+// four 32-lane quarters of tensor memory
+static_assert(kTConvWarps * 32 == 2 * kTRows, "converter threads: two per row");
+// the accumulator banks: 4 x 2 slots, 2 x 4 slots, 1 x kTSlots slots
+static_assert(4 * 2 * kTSlotCols <= kTTmemCols && 2 * 4 * kTSlotCols <= kTTmemCols &&
+                  kTSlots * kTSlotCols <= kTTmemCols,
+              "accumulator banks exceed the tensor-memory allocation");
+// one A_pack box per lane of its producer warp: two halves x two 16-row groups
+static_assert(4 * kTSlots <= 32, "A_pack boxes of a stage exceed a warp");
+// the widest sweep still fits two bf16 slices, two A_pack stages and one Xq
+// stage; the slots' sums (16 KB each) and the staged tables fit as well
+static_assert(kTABufs * kTABytes + 2 * kTSlots * kTSlotBytes + kTXSub * kTXBytes <=
+                  kTSmem - 1024,
+              "shared-memory layout of the widest sweep");
+static_assert(kTSlots * kTRows * 128 <= kTSmem - 1024 &&
+                  static_cast<int>(sizeof(int32_t)) * (4 * kTTab + 1) <= kTSmem - 1024,
+              "sums or tables exceed shared memory");
+
 // K splits for M tokens: about kTTargetCtas CTAs in all, at most a portable
 // cluster, and at least kTMinSlicesPerSplit K slices per split.
 static inline int tc_shrink_splits(int64_t M) {
@@ -391,7 +409,7 @@ struct ShrinkCtl {
   uint64_t xfull[kTMaxXStages], xempty[kTMaxXStages];  // Xq ring: TMA -> converters
   uint64_t pfull[kTMaxPStages], pempty[kTMaxPStages];  // A_pack ring: TMA -> MMAs
   uint64_t afull[kTABufs], aempty[kTABufs];            // bf16 slices: converters <-> MMAs
-  uint64_t done, tfree, drain;                     // accumulators ready / read / MMAs retired
+  uint64_t done, drain;                            // accumulators ready / MMAs retired
   uint32_t tmem_base;
   int abort, npass;
   int ad[kTRows], off[kTRows], rank[kTRows], groups[kTRows];
@@ -473,7 +491,6 @@ __global__ void __launch_bounds__(kTThreads, 1) lora_shrink_tc_kernel(
       mbar_init(&ctl.aempty[i], 1);
     }
     mbar_init(&ctl.done, 1);
-    mbar_init(&ctl.tfree, 4);
     mbar_init(&ctl.drain, 1);
     ctl.abort = 0;
     fence_mbar_init();
