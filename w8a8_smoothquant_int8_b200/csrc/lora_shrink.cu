@@ -441,6 +441,11 @@ __device__ __forceinline__ void share_rows(int q, int ns, int &lo, int &hi) {
   hi = (q + 1) * kTRows / ns;
 }
 
+// kRaw: T = X·A'ᵀ from the bf16 activations themselves (x_scale unused): each
+// X slice is already the MMA's bf16 operand, so there is no conversion; an X
+// stage is one slice (two 64-wide halves of 128 rows, 256 bytes of a row) and
+// is released by the MMAs that read it.
+template <bool kRaw>
 __global__ void __launch_bounds__(kTThreads, 1) lora_shrink_tc_kernel(
     const __grid_constant__ CUtensorMap tm_xq, const __grid_constant__ CUtensorMap tm_a,
     const float *__restrict__ x_scale, int64_t M, int64_t K,
@@ -480,7 +485,8 @@ __global__ void __launch_bounds__(kTThreads, 1) lora_shrink_tc_kernel(
   if (threadIdx.x == 0) {
     for (int i = 0; i < kTMaxXStages; ++i) {
       mbar_init(&ctl.xfull[i], 1);
-      mbar_init(&ctl.xempty[i], kTConvWarps);  // every converter warp has read the slice
+      // every converter warp has read the slice (raw: the MMAs that read it)
+      mbar_init(&ctl.xempty[i], kRaw ? 1 : kTConvWarps);
     }
     for (int i = 0; i < kTMaxPStages; ++i) {
       mbar_init(&ctl.pfull[i], 1);
@@ -555,8 +561,9 @@ __global__ void __launch_bounds__(kTThreads, 1) lora_shrink_tc_kernel(
     }
   }
   __syncthreads();
-  // the tokens' codes and scales come from the preceding kernel (programmatic
-  // dependent launch: everything above overlapped its tail)
+  // the tokens' codes and scales (raw: activations) may come from the
+  // preceding kernel (programmatic dependent launch: everything above
+  // overlapped its tail)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int npass = ctl.npass;
   const int nsweep = (npass + kTSlots - 1) / kTSlots;
@@ -565,14 +572,16 @@ __global__ void __launch_bounds__(kTThreads, 1) lora_shrink_tc_kernel(
   // A_pack ring (released when the MMAs that read it complete), then the Xq
   // ring (released as soon as a slice is converted, so more of its stages
   // are in flight than in one ring of both)
-  const int nab = kTABufs;
+  constexpr int kXSlices = kRaw ? 1 : kTXSub;        // K slices per X stage
+  constexpr int kXStageBytes = kRaw ? kTABytes : kTXSub * kTXBytes;
+  const int nab = kRaw ? 0 : kTABufs;
   const int pstage_bytes = slots_max * kTSlotBytes;
   const int pstages = slots_max <= 2 ? 3 : 2;
-  int xstages = (kTSmem - 1024 - nab * kTABytes - pstages * pstage_bytes) / (kTXSub * kTXBytes);
+  int xstages = (kTSmem - 1024 - nab * kTABytes - pstages * pstage_bytes) / kXStageBytes;
   xstages = xstages > kTMaxXStages ? kTMaxXStages : xstages;
   uint8_t *abuf = base;                                 // nab bf16 slices
   uint8_t *pring = base + nab * kTABytes;               // A_pack slots of each stage
-  uint8_t *xring = pring + pstages * pstage_bytes;      // int8 slices
+  uint8_t *xring = pring + pstages * pstage_bytes;      // int8 (raw: bf16) slices
   // independent accumulator banks: the K steps of a slice go to different
   // banks, so consecutive MMAs do not wait on each other; summed at the end
   const int nbank = (slots_max <= 2) ? 4 : ((slots_max <= 4) ? 2 : 1);
@@ -586,18 +595,19 @@ __global__ void __launch_bounds__(kTThreads, 1) lora_shrink_tc_kernel(
     for (int sw = 0; sw < nsweep; ++sw) {
       if (lane == 0) {
         if (sw == 0) prefetch_tmap(&tm_xq);
-        for (int c = c0; c < c1; c += kTXSub) {
+        for (int c = c0; c < c1; c += kXSlices) {
           if (*abort_flag || !mbar_wait(&ctl.xempty[st], ph ^ 1u, timeout_ns, abort_flag)) {
             *abort_flag = 1;
             record_device_error(SQ_ERR_DEVICE_TIMEOUT);
             break;
           }
-          // the stage's slices back to back: adjacent 128-byte pieces of each row
-          const int nsub = min(kTXSub, c1 - c);
-          mbar_arrive_expect_tx(&ctl.xfull[st], static_cast<uint32_t>(nsub * kTXBytes));
-          for (int u = 0; u < nsub; ++u)
-            tma_load_2d(xring + (st * kTXSub + u) * kTXBytes, &tm_xq, &ctl.xfull[st],
-                        (c + u) * kTK, static_cast<int32_t>(row0));
+          // 16 KB boxes back to back: adjacent 128-byte pieces of each row
+          // (int8: whole slices; raw: the two 64-wide halves of one slice)
+          const int nbox = kRaw ? 2 : min(kTXSub, c1 - c);
+          mbar_arrive_expect_tx(&ctl.xfull[st], static_cast<uint32_t>(nbox * kTXBytes));
+          for (int u = 0; u < nbox; ++u)
+            tma_load_2d(xring + st * kXStageBytes + u * kTXBytes, &tm_xq, &ctl.xfull[st],
+                        kRaw ? c * kTK + 64 * u : (c + u) * kTK, static_cast<int32_t>(row0));
           ++issued;
           if (++st == xstages) { st = 0; ph ^= 1u; }
         }
@@ -692,13 +702,15 @@ __global__ void __launch_bounds__(kTThreads, 1) lora_shrink_tc_kernel(
         tc_fence_after();  // the previous sweep's accumulators have been read
         bool ok = !*abort_flag;
         for (int c = c0; c < c1 && ok; ++c) {
-          if (!mbar_wait(&ctl.afull[b], bph, timeout_ns, abort_flag) ||
+          // the bf16 slice: converted (b counts them) or, raw, the X stage
+          // itself (b counts the X ring's stages)
+          if (!mbar_wait(kRaw ? &ctl.xfull[b] : &ctl.afull[b], bph, timeout_ns, abort_flag) ||
               !mbar_wait(&ctl.pfull[st], ph, timeout_ns, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(abuf + b * kTABytes);
+          const uint32_t a_addr = smem_u32(kRaw ? xring + b * kXStageBytes : abuf + b * kTABytes);
           const uint32_t s_addr = smem_u32(pring + st * pstage_bytes);
           // one MMA per K step for all slots of the sweep: their A_pack rows
           // are contiguous within each 64-wide half (a slot narrower than 32
@@ -713,10 +725,10 @@ __global__ void __launch_bounds__(kTThreads, 1) lora_shrink_tc_kernel(
                     sdesc_kmajor_sw128(s_addr + h * (slots_max * kTSlotCols * 128) + 32 * k16),
                     idesc, (c > c0 || kk >= nbank) ? 1u : 0u);
           }
-          mma_commit(&ctl.aempty[b]);
+          mma_commit(kRaw ? &ctl.xempty[b] : &ctl.aempty[b]);
           mma_commit(&ctl.pempty[st]);
           if (++st == pstages) { st = 0; ph ^= 1u; }
-          if (++b == nab) { b = 0; bph ^= 1u; }
+          if (++b == (kRaw ? xstages : nab)) { b = 0; bph ^= 1u; }
         }
         if (ok) {
           mma_commit(&ctl.done);
@@ -749,7 +761,7 @@ __global__ void __launch_bounds__(kTThreads, 1) lora_shrink_tc_kernel(
     for (int sw = 0; sw < nsweep; ++sw) {
       const int p0 = sw * kTSlots, np = min(kTSlots, npass - p0);
       bool ok = !*abort_flag;
-      for (int c = c0; c < c1 && ok; ++c) {
+      for (int c = c0; c < c1 && ok && !kRaw; ++c) {
         const int u = (c - c0) % kTXSub;  // slice of the Xq stage
         ok = (u != 0 ||
               __all_sync(0xffffffffu, mbar_wait(&ctl.xfull[st], ph, timeout_ns, abort_flag))) &&
@@ -850,7 +862,7 @@ __global__ void __launch_bounds__(kTThreads, 1) lora_shrink_tc_kernel(
               s8[4] += pv[u][1].x; s8[5] += pv[u][1].y; s8[6] += pv[u][1].z; s8[7] += pv[u][1].w;
             }
         }
-        const float xs = x_scale[row];
+        const float xs = kRaw ? 1.0f : x_scale[row];
 #pragma unroll
         for (int j = 0; j < 8; ++j) s8[j] = (cb + 8 * c8 + j < rank) ? xs * s8[j] : 0.f;
         store_t8(T_hi, T_lo, row * R + off + cb + 8 * c8, s8);
@@ -891,6 +903,7 @@ __global__ void __launch_bounds__(kTThreads, 1) lora_shrink_tc_kernel(
 
 // Clusters of `size` CTAs of the tensor-memory form that are resident at
 // once on the current device (asked of the runtime once per device and size).
+template <bool kRaw>
 static cudaError_t tc_clusters_resident(int size, int *out) {
   static std::atomic<int> cache[kMaxDevices][kTMaxSplit + 1];
   const int dev = current_device_index();
@@ -908,7 +921,7 @@ static cudaError_t tc_clusters_resident(int size, int *out) {
     attr.val.clusterDim.z = 1;
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, lora_shrink_tc_kernel, &cfg);
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, lora_shrink_tc_kernel<kRaw>, &cfg);
     if (e != cudaSuccess) return e;
     n = n > 0 ? n + 1 : 1;  // stored plus one: 0 means not asked yet
     cache[dev][size].store(n, std::memory_order_relaxed);
@@ -919,7 +932,9 @@ static cudaError_t tc_clusters_resident(int size, int *out) {
 
 // Launch of the tensor-memory form: 128-token blocks, K split over a cluster
 // of up to eight CTAs so that about one CTA per SM runs, all clusters at once.
-static cudaError_t launch_lora_shrink_tc(const int8_t *Xq, const float *x_scale, int64_t M,
+// X: Xq (int8) or, kRaw, the bf16 activations (x_scale unused).
+template <bool kRaw>
+static cudaError_t launch_lora_shrink_tc(const void *X, const float *x_scale, int64_t M,
                                          int64_t K, const uint16_t *A_pack,
                                          const int32_t *lora_offset, const int32_t *lora_rank,
                                          int n_adapters, int64_t R, const int32_t *seg_offsets,
@@ -932,14 +947,14 @@ static cudaError_t launch_lora_shrink_tc(const int8_t *Xq, const float *x_scale,
   const int most = nslices / kTMinSlicesPerSplit;  // keep at least a few slices per split
   if (nsplit > most) nsplit = most > 1 ? most : 1;
   static std::atomic<int> attr_set[kMaxDevices];
-  cudaError_t e = ensure_smem_optin(lora_shrink_tc_kernel, kTSmem, attr_set);
+  cudaError_t e = ensure_smem_optin(lora_shrink_tc_kernel<kRaw>, kTSmem, attr_set);
   if (e != cudaSuccess) return e;
   // the widest split whose clusters are all resident at once (one CTA per
   // SM: clusters of 3 or more CTAs leave SMs of a GPC unused, so fewer of
   // them fit than SMs / size)
   while (nsplit > 1) {
     int fit = 0;
-    e = tc_clusters_resident(nsplit, &fit);
+    e = tc_clusters_resident<kRaw>(nsplit, &fit);
     if (e != cudaSuccess) return e;
     if (fit >= nrb) break;
     --nsplit;
@@ -947,8 +962,12 @@ static cudaError_t launch_lora_shrink_tc(const int8_t *Xq, const float *x_scale,
   CUtensorMap tm_xq, tm_a;
   memset(&tm_xq, 0, sizeof tm_xq);
   memset(&tm_a, 0, sizeof tm_a);
-  if (!make_tmap(&tm_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, kTK, kTRows,
-                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+  const bool x_ok =
+      kRaw ? make_tmap(&tm_xq, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M, 64, kTRows,
+                       CU_TENSOR_MAP_SWIZZLE_128B)
+           : make_tmap(&tm_xq, X, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, kTK, kTRows,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!x_ok ||
       !make_tmap(&tm_a, A_pack, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, R, 64, 16))
     return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
@@ -965,7 +984,7 @@ static cudaError_t launch_lora_shrink_tc(const int8_t *Xq, const float *x_scale,
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, lora_shrink_tc_kernel, tm_xq, tm_a, x_scale, M, K, lora_offset,
+  return cudaLaunchKernelEx(&cfg, lora_shrink_tc_kernel<kRaw>, tm_xq, tm_a, x_scale, M, K, lora_offset,
                             lora_rank, n_adapters, R, seg_offsets, seg_adapter, S, nsplit, T_hi,
                             T_lo, mask, wait_timeout_ns());
 }
@@ -1035,8 +1054,9 @@ cudaError_t launch_lora_shrink(const int8_t *Xq, const float *x_scale, int64_t M
   // this one; K split over clusters fills the remaining SMs)
   const int nsm = sm_count_of_current_device();
   if (nsm > 0 && M >= static_cast<int64_t>(kTRows) * (nsm / 5))
-    return launch_lora_shrink_tc(Xq, x_scale, M, K, A_pack, lora_offset, lora_rank, n_adapters,
-                                 R, seg_offsets, seg_adapter, S, T_hi, T_lo, mask, st);
+    return launch_lora_shrink_tc<false>(Xq, x_scale, M, K, A_pack, lora_offset, lora_rank,
+                                        n_adapters, R, seg_offsets, seg_adapter, S, T_hi, T_lo,
+                                        mask, st);
   return launch_lora_shrink_t<false>(Xq, x_scale, M, K, A_pack, lora_offset, lora_rank,
                                      n_adapters, R, seg_offsets, seg_adapter, S, T_hi, T_lo, mask,
                                      st);
@@ -1049,6 +1069,12 @@ cudaError_t launch_lora_shrink_raw(const uint16_t *X, int64_t M, int64_t K,
                                    int64_t S, uint16_t *T_hi, uint16_t *T_lo,
                                    unsigned long long *mask, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
+  // the tensor-memory form from the same number of tokens as above
+  const int nsm = sm_count_of_current_device();
+  if (nsm > 0 && M >= static_cast<int64_t>(kTRows) * (nsm / 5))
+    return launch_lora_shrink_tc<true>(X, nullptr, M, K, A_pack, lora_offset, lora_rank,
+                                       n_adapters, R, seg_offsets, seg_adapter, S, T_hi, T_lo,
+                                       mask, st);
   return launch_lora_shrink_t<true>(X, nullptr, M, K, A_pack, lora_offset, lora_rank, n_adapters,
                                     R, seg_offsets, seg_adapter, S, T_hi, T_lo, mask, st);
 }
