@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(kShrinkThreads) lora_shrink_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Tensor-memory form (large M, quantized input).  The warp-level MMAs above
+// Tensor-memory form (large M; codes or, raw, bf16 input).  The warp-level MMAs above
 // run on the legacy tensor path, which on this GPU sustains only a few
 // hundred multiply-adds per clock per SM: at the largest workloads the form
 // above is bound by it (measured: the same ~1 us per 64-wide K slice per warp
