@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(kShrinkThreads) lora_shrink_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Tensor-memory form (large M; codes or, raw, bf16 input).  The warp-level MMAs above
+// Tensor-memory form (large M; codes, or raw bf16 input).  The warp-level MMAs above
 // run on the legacy tensor path, which on this GPU sustains only a few
 // hundred multiply-adds per clock per SM: at the largest workloads the form
 // above is bound by it (measured: the same ~1 us per 64-wide K slice per warp
@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(kShrinkThreads) lora_shrink_kernel(
 // on timing.  Output as in the form above.
 // ---------------------------------------------------------------------------
 constexpr int kTRows = 128;                     // tokens per CTA (the MMA's M)
-constexpr int kTK = 128;                        // K per stage (one 128-byte Xq row)
+constexpr int kTK = 128;                        // K per slice (128 bytes of an Xq row)
 constexpr int kTSlotCols = 32;                  // TMEM columns per slot
 constexpr int kTSlots = 5;                      // slots per sweep over K
 constexpr int kTTmemCols = 256;                 // >= kTSlots * kTSlotCols, a power of 2
